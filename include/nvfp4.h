@@ -1,0 +1,200 @@
+/*
+ * nvfp4.h — C ABI of libnvfp4.so, the NVFP4 W4A4 linear layer for sm_100a.
+ *
+ * Sources (web pages about "Why Gated DeltaNet Survives 4-Bit Quantization:
+ * NVFP4 W4A4 for the Recurrent Half of a Hybrid 27B LLM", arXiv 2609.04098):
+ *   [news]     "Qwen3.8-27B最激进4bit量化开源，权重显存暴降2.9倍！", sections 02
+ *              (NVFP4 量化格式) and 03 (Minima 模型构建);
+ *   [reading]  MessageDaily paper reading "minima-gdn-4bit-quantization",
+ *              section 一 (论文背景) and section 4.1;
+ *   [abstract] arXiv 2609.04098 abstract (English abstract).
+ *
+ * FORMAT (news §02; reading §一). A tensor X[rows][k] is stored as
+ *   - codes: 4-bit E2M1 values, row-major [rows][k/2] bytes, element 2j of a
+ *            row in the LOW nibble of byte j, element 2j+1 in the high nibble.
+ *            Code = sign*8 + m, m = 0..7 -> {0, 0.5, 1, 1.5, 2, 3, 4, 6}.
+ *   - sf:    one unsigned E4M3 block scale per 16 contiguous elements along k,
+ *            stored in the 128x4 swizzled layout (below).
+ *   - g:     one FP32 global scale per tensor (a device scalar).
+ * Dequantized value: val(code) * dec(sf) / g.
+ *
+ * CONVENTION (the pages name the three scales but give no formula; this is the
+ * convention the library fixes, evaluated in IEEE FP32 round-to-nearest-even):
+ *   amax = max |x| over the tensor (exact);  g = 2688 / amax  (2688 = 448*6);
+ *          g = 1 if amax == 0 or the quotient is not finite.
+ *   per 16-element block b:  t = amax_b / 6;  s = E4M3_rne_satfinite(t * g);
+ *   per element:  r = g / dec(s);  code = E2M1_rne_satfinite(x * r);
+ *                 if dec(s) == 0 every code of the block is a signed zero.
+ *   The sign of a code is the sign bit of x * r (so -0.0 and tiny negatives
+ *   encode as 0x8).
+ *
+ * SCALE-FACTOR LAYOUT ("128x4 swizzle"). With kb = k/16 blocks per row,
+ *   KB4 = ceil(kb/4)*4 and R128 = ceil(rows/128)*128, the buffer holds
+ *   R128*KB4 bytes (nvfp4_sf_bytes). Block (r, c) lives at byte
+ *     ((r/128)*(KB4/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4 + (c%4).
+ *   Each 512-byte atom covers 128 rows x 4 blocks; bytes for r >= rows or
+ *   c >= kb are zero. This is the layout the sm_100 block-scaled tensor-core
+ *   instruction consumes after a 32x128b tensor-memory copy.
+ *
+ * CONVENTIONS OF THE ABI
+ *   - Every pointer named "device" is CUDA global memory of the current device.
+ *     The caller owns every buffer; the library keeps no per-call state.
+ *   - Every compute call is asynchronous on the given stream; argument checks
+ *     are synchronous and return a status before anything is launched.
+ *   - Global scales stay on the device: no call synchronises with the host.
+ *   - NaN / Inf inputs are outside the contract.
+ *   - No C++ exception crosses this boundary.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Opaque CUDA stream handle (cudaStream_t); NULL is the legacy default stream. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,  /* null pointer, negative/zero size, bad enum   */
+  NVFP4_ERR_UNSUPPORTED = 2,  /* shape outside what the kernels implement     */
+  NVFP4_ERR_MISALIGNED = 3,   /* pointer or pitch alignment rule broken       */
+  NVFP4_ERR_CUDA = 4,         /* a CUDA runtime / driver call failed          */
+  NVFP4_ERR_TIMEOUT = 5       /* a kernel's bounded wait expired (fault word) */
+} nvfp4_status;
+
+/* Human-readable name of a status. Never NULL. */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/* Bytes of the swizzled scale-factor buffer of a [rows][k] tensor:
+ * ceil(rows/128)*128 * ceil(k/64)*4.  Returns 0 if rows < 0, k <= 0 or
+ * k % 16 != 0. */
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k);
+
+/* Workspace bytes nvfp4_quantize needs in dynamic-global mode (per-CTA
+ * partial maxima). Static mode needs none. */
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
+
+/*
+ * nvfp4_quantize — activation / weight quantization (news §02: E2M1 values,
+ * one E4M3 scale per 16 elements, one FP32 global scale; W4A4 quantizes both
+ * weights and activations, reading §4.1 / news §03).
+ *
+ *   x          device, bf16 [rows][ldx] (only the first k of each row are
+ *              read); 16-byte aligned, ldx % 8 == 0, ldx >= k.
+ *   rows       >= 0 (0 writes nothing but global_out).
+ *   k          > 0, k % 16 == 0.
+ *   global_in  device FP32 scalar or NULL. NULL => dynamic mode: amax over x,
+ *              g = 2688/amax (two kernels: an amax pass, then the quantizer).
+ *              Non-NULL => static (calibrated) mode: g = *global_in as given;
+ *              block scales may then saturate at 448 and codes at +-6.
+ *   codes      device, [rows][k/2] bytes, row pitch k/2; 4-byte aligned.
+ *   sf         device, nvfp4_sf_bytes(rows, k) bytes, 16-byte aligned; every
+ *              byte is written (padding = 0).
+ *   global_out device FP32 scalar: receives g. May equal global_in.
+ *   workspace  device scratch of >= nvfp4_quantize_workspace_bytes(rows,k)
+ *              bytes, 16-byte aligned (dynamic mode only; may be NULL in
+ *              static mode). Contents need no initialisation.
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED (k % 16), CUDA (launch).
+ */
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
+                            const float* global_in, uint8_t* codes, uint8_t* sf,
+                            float* global_out, void* workspace,
+                            size_t workspace_bytes, nvfp4_stream_t stream);
+
+/* Workspace bytes nvfp4_gemm needs (0 for every shape the current kernels
+ * handle; kept so callers need not change when split-K arrives). */
+size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/*
+ * nvfp4_gemm — W4A4 block-scaled GEMM on the 4-bit tensor cores (news §02:
+ * "hardware-native 4-bit tensor cores"):
+ *   Y[i][j] = (1 / (g_a * g_b)) * sum_k val(A)[i][k]*dec(sfA)[i][k/16]
+ *                                      * val(B)[j][k]*dec(sfB)[j][k/16]
+ * i.e. Y = dequant(A) @ dequant(B)^T, accumulated in FP32.
+ *
+ *   a_codes, a_sf, a_global  A = activations, [m][k] NVFP4 as nvfp4_quantize
+ *                            writes it; a_global is a device FP32 scalar.
+ *   b_codes, b_sf, b_global  B = weights, [n][k] NVFP4 (row j = output j).
+ *   y        device, [m][ldy] of bf16 (y_dtype 0) or fp32 (y_dtype 1);
+ *            16-byte aligned; ldy >= n; ldy*elem % 16 == 0.
+ *   m, n     >= 1.   k: k % 32 == 0 (TMA row pitch k/2 must be a multiple of
+ *            16 bytes) and k >= 32.
+ *   a_codes, b_codes: 16-byte aligned. a_sf, b_sf: 16-byte aligned.
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
+ */
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
+                        const float* a_global, const uint8_t* b_codes,
+                        const uint8_t* b_sf, const float* b_global, void* y,
+                        int y_dtype, int64_t ldy, int64_t m, int64_t n,
+                        int64_t k, void* workspace, size_t workspace_bytes,
+                        nvfp4_stream_t stream);
+
+/*
+ * nvfp4_fuse_group_scales — global-scale repair of a fused module group
+ * (news §03: a serving kernel fuses several GDN linear layers into one GEMM;
+ * taking the group's largest global scale without rescaling the block scales
+ * distorts the weights, so the group is brought onto one global scale and the
+ * ratio folded into the E4M3 block scales; abstract: "global-scale mismatch").
+ *
+ *   g*   = min_i g_i  (the global of the module with the largest amax, i.e.
+ *          the global the concatenated tensor would get; every ratio <= 1 so
+ *          no block scale can saturate).
+ *   r_i  = g* / g_i (FP32 RN);  s' = E4M3_rne_satfinite(dec(s) * r_i) (FP32 RN
+ *          multiply);  codes are unchanged.
+ * Out of place: module i's scale factors, as nvfp4_quantize wrote them for its
+ * own [rows_i][k] tensor, are rescaled and written into the swizzled layout
+ * of the row-concatenated [sum rows_i][k] tensor (modules in argument order;
+ * atoms shared by two modules are filled from both; padding = 0). The codes
+ * of the concatenated tensor are simply the modules' code rows back to back
+ * (quantize module i straight into the fused code buffer at row offset
+ * sum_{j<i} rows_j).
+ *
+ *   n_modules        1..16.
+ *   rows_per_module  HOST array [n_modules], each >= 1.
+ *   k                > 0, k % 16 == 0 (common to all modules).
+ *   sf_modules       HOST array [n_modules] of device pointers, each
+ *                    nvfp4_sf_bytes(rows_i, k) bytes, 4-byte aligned.
+ *   globals_in       device FP32 [n_modules]: the modules' own g_i.
+ *   sf_fused         device, nvfp4_sf_bytes(sum rows_i, k) bytes, 16-byte
+ *                    aligned; must not overlap any sf_modules buffer.
+ *   global_out       device FP32 scalar: receives g*.
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
+ */
+nvfp4_status nvfp4_fuse_group_scales(int n_modules,
+                                     const int64_t* rows_per_module, int64_t k,
+                                     const uint8_t* const* sf_modules,
+                                     const float* globals_in, uint8_t* sf_fused,
+                                     float* global_out, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_silu_mul — the gated-MLP activation between the gate_up and the down
+ * projection of a W4A4 MLP (not specified by the pages, which only state that
+ * every linear layer is quantized, news §03): h = bf16_rn(silu(gate) * up),
+ * silu(z) = z / (1 + exp(-z)), in FP32.
+ *   y   device bf16 [m][ldy]; gate = columns [0, n), up = columns [n, 2n).
+ *   h   device bf16 [m][ldh].
+ *   n % 8 == 0, ldy % 8 == 0, ldh % 8 == 0, both pointers 16-byte aligned.
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
+ */
+nvfp4_status nvfp4_silu_mul(const void* y, int64_t m, int64_t n, int64_t ldy,
+                            void* h, int64_t ldh, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_read_fault — every mbarrier wait in the GEMM kernel is bounded; on
+ * expiry the kernel records a nonzero fault word, stops issuing work and
+ * returns instead of hanging. This call synchronises `stream`, copies the
+ * fault word to *fault_out (0 = none) and clears it. Returns NVFP4_ERR_TIMEOUT
+ * if the word was nonzero, else NVFP4_OK (or NVFP4_ERR_CUDA).
+ */
+nvfp4_status nvfp4_read_fault(nvfp4_stream_t stream, uint32_t* fault_out);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* NVFP4_H_ */
