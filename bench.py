@@ -1,0 +1,521 @@
+"""Benchmark of the NVFP4 W4A4 linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl reference]
+
+A step is one pass of the hot path over one batch of seeded synthetic input:
+activation quantization (amax pass + quantizer, dynamic global scale) and the
+block-scaled FP4 GEMM against weights quantized beforehand (weights are
+offline in a W4A4 checkpoint). Workloads:
+  outlier    X 8192x5120 (8 channels x50) @ W 5120x5120        (default)
+  gdn_fused  X 8192x5120 @ fused qkv|z|a|b 12384x5120 (fold done offline)
+  mlp32k     X 32768x5120 -> gate_up 34816 -> silu*mul -> requant -> down 5120
+Metric: TFLOP/s of the whole step (2*M*N*K per GEMM over quantize + GEMM
+time), with the GEMM's fraction of the dense FP4 tensor peak and the
+quantizer's GB/s alongside. Inputs stay resident in HBM; L2 (126 MB) is
+flushed by a 256 MiB write before every timed step, outside the timed events.
+
+Multi-GPU (torchrun): every rank runs the same step on its own batch (weak
+scaling, no collective on the data path); the per-rank device time is
+reduced with MAX and the value counts all ranks' FLOPs.
+
+--impl reference times the CPU oracle (the plain reference this library is
+checked against) on the host cores, on a bounded row sample per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 W4A4 GEMM TFLOPS incl. act quant, % dense FP4 peak; quant GB/s"
+FP4_SPEC_TFLOPS = 9000.0          # B200 dense FP4, public spec
+HBM_SPEC_GBS = 8000.0
+QUANT_BYTES_PER_ELEM = 2.5625     # read bf16 + write 0.5 code + 1/16 scale
+AMAX_BYTES_PER_ELEM = 2.0
+L2_FLUSH_BYTES = 256 << 20
+
+
+def peaks():
+    """Roofline denominators: the measured peaks if present."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        mp = json.load(open(path))
+        return {"hbm_gbs": float(mp["hbm_gbs"]), "bf16_tflops": float(mp["bf16_tflops"]),
+                "bf16_tflops_sustained": float(mp.get("bf16_tflops_sustained", mp["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------ clocks --
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.samples = []
+        self.proc = None
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        rows = [s for (t, s) in self.samples if t0 <= t <= t1]
+        window = "timed region"
+        if len(rows) < 3:  # timed region shorter than a few sample periods
+            rows = [s for (_, s) in self.samples]
+            window = "whole run (timed region shorter than 3 samples)"
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            f = [x.strip() for x in r.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm), "window": window}
+
+
+# --------------------------------------------------------------- workloads --
+
+def make_workload(name: str, rank: int):
+    """Device-resident inputs and pre-quantized weights of one workload."""
+    from nvfp4_w4a4_quantized_elem_b200 import nvfp4, workloads as wl
+    if name == "outlier":
+        cfg = wl.outlier()
+        cfg.x_seed = wl.SEED_X + 1000 * rank
+        x = cfg.x().cuda()
+        W = nvfp4.quantize(cfg.w().cuda())
+        gemms = [(cfg.m, cfg.n, cfg.k)]
+        desc = (f"outlier: X {cfg.m}x{cfg.k} bf16 ~N(0,1) with 8 channels x50, "
+                f"W {cfg.n}x{cfg.k} ~N(0,0.02) NVFP4; quantize X + W4A4 GEMM -> bf16")
+        return dict(x=x, W=W, gemms=gemms, desc=desc, kind="linear", m=cfg.m, n=cfg.n, k=cfg.k)
+    if name == "gdn_fused":
+        cfg = wl.gdn_fused()
+        x = wl.gaussian_bf16(cfg.m, cfg.k, 1.0, wl.SEED_X + 1000 * rank).cuda()
+        mods = [nvfp4.quantize(w.cuda()) for w in cfg.weights()]
+        W = nvfp4.fuse_group(mods)
+        desc = (f"gdn_fused: X {cfg.m}x{cfg.k} @ fused qkv|z|a|b {cfg.n}x{cfg.k} "
+                "(per-module globals folded offline); quantize X + one fused GEMM")
+        return dict(x=x, W=W, gemms=[(cfg.m, cfg.n, cfg.k)], desc=desc, kind="linear",
+                    m=cfg.m, n=cfg.n, k=cfg.k)
+    if name == "mlp32k":
+        cfg = wl.mlp32k()
+        x = cfg.x().cuda()
+        Wgu = nvfp4.quantize(cfg.w_gate_up().cuda())
+        Wd = nvfp4.quantize(cfg.w_down().cuda())
+        desc = (f"mlp32k: X {cfg.m}x{cfg.d} -> gate_up {2 * cfg.ffn}x{cfg.d} -> silu*mul -> "
+                f"requant -> down {cfg.d}x{cfg.ffn}")
+        return dict(x=x, Wgu=Wgu, Wd=Wd, gemms=[(cfg.m, 2 * cfg.ffn, cfg.d), (cfg.m, cfg.d, cfg.ffn)],
+                    desc=desc, kind="mlp", m=cfg.m, n=cfg.d, k=cfg.d, ffn=cfg.ffn)
+    raise SystemExit(f"unknown workload {name}")
+
+
+class Step:
+    """One pass of the hot path with CUDA events between the phases."""
+
+    def __init__(self, wk, stream):
+        from nvfp4_w4a4_quantized_elem_b200 import nvfp4
+        self.nv = nvfp4
+        self.wk = wk
+        self.s = stream
+        dev = wk["x"].device
+        m, k = wk["x"].shape
+        self.A = nvfp4.NVFP4Tensor.empty(m, k, dev)
+        self.ws = torch.empty(nvfp4.quantize_workspace_bytes(m, k), dtype=torch.uint8, device=dev)
+        if wk["kind"] == "linear":
+            self.y = torch.empty((m, wk["W"].rows), dtype=torch.bfloat16, device=dev)
+        else:
+            ffn = wk["ffn"]
+            self.ygu = torch.empty((m, 2 * ffn), dtype=torch.bfloat16, device=dev)
+            self.h = torch.empty((m, ffn), dtype=torch.bfloat16, device=dev)
+            self.H = nvfp4.NVFP4Tensor.empty(m, ffn, dev)
+            self.y = torch.empty((m, wk["n"]), dtype=torch.bfloat16, device=dev)
+        self.launches = 3 if wk["kind"] == "linear" else 9
+
+    def run(self, ev=None, x=None):
+        nv, wk, s = self.nv, self.wk, self.s
+        x = wk["x"] if x is None else x
+        rec = (lambda i: ev[i].record(s)) if ev is not None else (lambda i: None)
+        rec(0)
+        nv.quantize(x, out=self.A, workspace=self.ws, stream=s)
+        rec(1)
+        if wk["kind"] == "linear":
+            nv.gemm(self.A, wk["W"], out=self.y, stream=s)
+            rec(2)
+        else:
+            nv.gemm(self.A, wk["Wgu"], out=self.ygu, stream=s)
+            rec(2)
+            nv.silu_mul(self.ygu, out=self.h, stream=s)
+            nv.quantize(self.h, out=self.H, workspace=self.ws, stream=s)
+            rec(3)
+            nv.gemm(self.H, wk["Wd"], out=self.y, stream=s)
+            rec(4)
+        return self.y
+
+
+def gemm_source_hash() -> str:
+    p = os.path.join(ROOT, "nvfp4_w4a4_quantized_elem_b200", "csrc", "gemm_sm100.cuh")
+    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+
+
+def dram_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
+    taken on the current GEMM source; else None."""
+    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    try:
+        d = json.load(open(p))
+        e = d.get(workload)
+        if e and e.get("gemm_source_sha256_16") == gemm_source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ GPU arm --
+
+def run_gpu(args):
+    from nvfp4_w4a4_quantized_elem_b200 import build as nb, nvfp4
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        nb.build()
+    if dist is not None:
+        dist.barrier()
+    nvfp4.lib()
+
+    wk = make_workload(args.workload, rank)
+    stream = torch.cuda.Stream()
+    step = Step(wk, stream)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
+    flops = sum(2 * m * n * k for (m, n, k) in wk["gemms"])
+    nph = 3 if wk["kind"] == "linear" else 5
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.fill_(1)
+            step.run()
+    stream.synchronize()
+    assert nvfp4.read_fault(stream) == 0
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nph)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    with torch.cuda.stream(stream):
+        for i in range(args.steps):
+            flush.fill_(i & 0xFF)  # evict L2 outside the timed events
+            step.run(events[i])
+    stream.synchronize()
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if dist is not None:
+        dist.barrier()
+    # one extra second of the same step for the clock record if the timed
+    # region was shorter than a few sample periods (not part of any number)
+    if t1 - t0 < 1.0:
+        with torch.cuda.stream(stream):
+            end = time.time() + 1.0
+            while time.time() < end:
+                for _ in range(20):
+                    step.run()
+                stream.synchronize()
+    sampler.stop()
+    clocks = sampler.summary(t0, t1)
+
+    step_ms = [events[i][0].elapsed_time(events[i][nph - 1]) for i in range(args.steps)]
+    quant_ms = [events[i][0].elapsed_time(events[i][1]) for i in range(args.steps)]
+    gemm_ms = [events[i][1].elapsed_time(events[i][2]) for i in range(args.steps)]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = flops * world / (ms_per_step * 1e-3) / 1e12
+
+    # component figures on this rank
+    m, k = wk["x"].shape
+    gemm_avg_ms = statistics.mean(gemm_ms)
+    q_avg_ms = statistics.mean(quant_ms)
+    pk = peaks()
+    fp4_peak = 4.0 * pk["bf16_tflops"]
+    gemm0 = wk["gemms"][0]
+    gemm_tflops = 2 * gemm0[0] * gemm0[1] * gemm0[2] / (gemm_avg_ms * 1e-3) / 1e12
+
+    # quantizer alone (static global: no amax pass), same input, L2 flushed
+    gstatic = step.A.global_scale.clone()
+    qev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(20)]
+    with torch.cuda.stream(stream):
+        for e0, e1 in qev:
+            flush.fill_(3)
+            e0.record(stream)
+            nvfp4.quantize(wk["x"], global_scale=gstatic, out=step.A, stream=stream)
+            e1.record(stream)
+    stream.synchronize()
+    qstatic_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in qev)
+    amax_ms = max(q_avg_ms - qstatic_ms, 1e-6)
+    elems = m * k
+    quant_gbs = elems * QUANT_BYTES_PER_ELEM / (qstatic_ms * 1e-3) / 1e9
+    amax_gbs = elems * AMAX_BYTES_PER_ELEM / (amax_ms * 1e-3) / 1e9
+
+    e2e = measure_e2e(step, wk, stream, flops, args)
+    if dist is not None:
+        t = torch.tensor([e2e["ms_per_step"]], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e["ms_per_step"] = float(t.item())
+        e2e["value"] = flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12
+
+    assert nvfp4.read_fault(stream) == 0
+    traffic = dram_traffic(args.workload)
+    out = {
+        "metric": METRIC,
+        "value": round(value, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "e2m1*e2m1 (e4m3 block scales) -> f32 acc -> bf16",
+        "data": "synthetic (seeded Gaussian, shapes of a 27B hybrid model's projections)",
+        "config": {"workload": wk["desc"], "gemms_mnk": wk["gemms"],
+                   "l2": "flushed (256 MiB write) before every timed step, outside the events",
+                   "parallelism": f"replicas x{world} (independent batches, no collective)"},
+        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
+                     "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
+                     "frac": round(gemm_tflops / fp4_peak, 4),
+                     "traffic": traffic,
+                     "kernel": "nvfp4::gemm::gemm_kernel",
+                     "peak_source": f"4 x bf16 burst of {pk['source']} ({pk['bf16_tflops']} TF/s; "
+                                    "4 = nominal FP4/BF16 dense ratio)",
+                     "frac_of_fp4_spec_9000": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
+                     "algorithmic_flops_per_launch": 2 * gemm0[0] * gemm0[1] * gemm0[2]},
+        "components": {
+            "quantize_ms": round(q_avg_ms, 5), "gemm_ms": round(gemm_avg_ms, 5),
+            "quantizer_alone_ms": round(qstatic_ms, 5), "amax_ms_est": round(amax_ms, 5),
+            "quant_gbs": round(quant_gbs, 1),
+            "quant_frac_hbm": round(quant_gbs / pk["hbm_gbs"], 4),
+            "amax_gbs": round(amax_gbs, 1),
+            "hbm_peak_gbs": pk["hbm_gbs"],
+            "quant_bytes_per_elem": QUANT_BYTES_PER_ELEM,
+        },
+        "e2e": {"value": round(e2e["value"], 2), "unit": "TFLOP/s",
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                "ms_per_step": round(e2e["ms_per_step"], 4)},
+        "gpu_launches": step.launches * args.steps,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def measure_e2e(step, wk, stream, flops, args):
+    """Through the public API with host buffers: each step copies X from
+    pinned host memory, runs the hot path, copies Y back to pinned memory."""
+    x_host = wk["x"].cpu().pin_memory()
+    y = step.y
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    x_dev = torch.empty_like(wk["x"])
+    n = max(3, min(args.steps, 20))
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n)]
+    with torch.cuda.stream(stream):
+        for _ in range(2):
+            x_dev.copy_(x_host, non_blocking=True)
+            step.run(x=x_dev)
+            y_host.copy_(y, non_blocking=True)
+        for e0, e1 in evs:
+            e0.record(stream)
+            x_dev.copy_(x_host, non_blocking=True)
+            step.run(x=x_dev)
+            y_host.copy_(y, non_blocking=True)
+            e1.record(stream)
+    stream.synchronize()
+    ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+    return {"value": flops / (ms * 1e-3) / 1e12, "ms_per_step": ms,
+            "h2d": x_host.numel() * x_host.element_size(),
+            "d2h": y_host.numel() * y_host.element_size()}
+
+
+# ------------------------------------------------------------ CPU oracle arm --
+
+def oracle_sample_step(orc, wk_cpu, rows):
+    """One bounded sample of the step on the CPU oracle: quantize `rows` rows
+    of X (dynamic global over the sample) and their FP64 GEMM rows."""
+    import numpy as np
+    xs = wk_cpu["x_bits"][:rows]
+    qa = orc.quantize(np.ascontiguousarray(xs))
+    if wk_cpu["kind"] == "linear":
+        return orc.gemm(qa, wk_cpu["qw"])
+    y = orc.gemm(qa, wk_cpu["qgu"])
+    yb = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    h = orc.silu_mul(yb)
+    return orc.gemm(orc.quantize(h), wk_cpu["qd"])
+
+
+def oracle_workload(name):
+    import numpy as np
+    import oracle as orc
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    if name == "outlier":
+        cfg = wl.outlier()
+        return orc, dict(kind="linear", x_bits=bits(cfg.x(rows=1024)), qw=orc.quantize(bits(cfg.w())),
+                         flops_per_row=2 * cfg.n * cfg.k)
+    if name == "gdn_fused":
+        cfg = wl.gdn_fused()
+        mods = [orc.quantize(bits(w)) for w in cfg.weights()]
+        return orc, dict(kind="linear", x_bits=bits(cfg.x()[:1024]), qw=orc.fuse_group(mods),
+                         flops_per_row=2 * cfg.n * cfg.k)
+    cfg = wl.mlp32k()
+    return orc, dict(kind="mlp", x_bits=bits(cfg.x(rows=1024)),
+                     qgu=orc.quantize(bits(cfg.w_gate_up())), qd=orc.quantize(bits(cfg.w_down())),
+                     flops_per_row=2 * (2 * cfg.ffn) * cfg.d + 2 * cfg.d * cfg.ffn)
+
+
+def cpu_baseline(name, budget_s=15.0, rows=128):
+    orc, w = oracle_workload(name)
+    oracle_sample_step(orc, w, 8)  # warm (builds/loads the oracle)
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle_sample_step(orc, w, rows)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s or reps >= 50:
+            break
+    tflops = w["flops_per_row"] * rows * reps / el / 1e12
+    return {"value": tflops, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+            "sample": f"{reps} x ({rows} rows of X: oracle quantize + FP64 GEMM vs the full "
+                      f"pre-quantized weights), {el:.1f} s of host time, scaled per FLOP"}
+
+
+def run_reference(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    orc, w = oracle_workload(args.workload)
+    rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample_step(orc, w, 8)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle_sample_step(orc, w, rows)
+        times.append(time.perf_counter() - t0)
+    ms = 1e3 * statistics.mean(times)
+    value = w["flops_per_row"] * rows / (ms * 1e-3) / 1e12
+    wk_desc = {"outlier": "outlier: X 8192x5120 (8 channels x50) @ W 5120x5120",
+               "gdn_fused": "gdn_fused: X 8192x5120 @ fused 12384x5120",
+               "mlp32k": "mlp32k: X 32768x5120 -> 34816 -> 17408 -> 5120"}[args.workload]
+    out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+           "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "f64 (oracle)", "data": "synthetic",
+           "config": {"workload": wk_desc, "sample_rows_per_step": rows},
+           "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": os.cpu_count(),
+                            "kind": "oracle",
+                            "sample": f"{rows} rows of X per step: oracle quantize + FP64 GEMM"},
+           "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="outlier", choices=["outlier", "gdn_fused", "mlp32k"])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=64)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,351 @@
+// nvfp4_api.cu — the C ABI of libnvfp4.so (declared in include/nvfp4.h).
+//
+// One translation unit: it includes every kernel header, validates arguments
+// on the host (returning a status before anything is launched), builds the
+// TMA descriptors of the GEMM and launches on the caller's stream. Nothing is
+// allocated and no call synchronises with the host except nvfp4_read_fault.
+#include "nvfp4.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "fold.cuh"
+#include "gemm_sm100.cuh"
+#include "quant.cuh"
+#include "silu_mul.cuh"
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  int sms = 0;
+  bool gemm_smem_set = false;
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nvfp4_status current_device(int* dev, DeviceState** st) {
+  if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& s = g_dev[*dev];
+  if (s.sms == 0) {
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess ||
+        sms <= 0) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    s.sms = sms;
+  }
+  *st = &s;
+  return NVFP4_OK;
+}
+
+nvfp4_status get_encoder(PFN_cuTensorMapEncodeTiled_v12000* fn) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (g_encode == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || p == nullptr) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  *fn = g_encode;
+  return NVFP4_OK;
+}
+
+nvfp4_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+}  // namespace
+
+extern "C" {
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "NVFP4_OK";
+    case NVFP4_ERR_INVALID_ARG: return "NVFP4_ERR_INVALID_ARG";
+    case NVFP4_ERR_UNSUPPORTED: return "NVFP4_ERR_UNSUPPORTED";
+    case NVFP4_ERR_MISALIGNED: return "NVFP4_ERR_MISALIGNED";
+    case NVFP4_ERR_CUDA: return "NVFP4_ERR_CUDA";
+    case NVFP4_ERR_TIMEOUT: return "NVFP4_ERR_TIMEOUT";
+  }
+  return "NVFP4_ERR_UNKNOWN";
+}
+
+size_t nvfp4_sf_bytes(int64_t rows, int64_t k) {
+  if (rows < 0 || k <= 0 || k % 16 != 0) return 0;
+  return static_cast<size_t>(ceil_div(rows, 128) * 128) * static_cast<size_t>(ceil_div(k, 64) * 4);
+}
+
+size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k) {
+  (void)rows;
+  (void)k;
+  return static_cast<size_t>(nvfp4::quant::kMaxPartials) * sizeof(float);
+}
+
+nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
+                            const float* global_in, uint8_t* codes, uint8_t* sf,
+                            float* global_out, void* workspace, size_t workspace_bytes,
+                            nvfp4_stream_t stream) {
+  using namespace nvfp4::quant;
+  if (rows < 0 || k <= 0 || global_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED;
+  if (rows > 0 && (x == nullptr || codes == nullptr || sf == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (ldx < k) return NVFP4_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(codes, 4) || !aligned(sf, 16) ||
+      !aligned(global_out, 4))
+    return NVFP4_ERR_MISALIGNED;
+  const bool dynamic = (global_in == nullptr);
+  if (dynamic) {
+    if (workspace == nullptr || workspace_bytes < nvfp4_quantize_workspace_bytes(rows, k))
+      return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return NVFP4_ERR_MISALIGNED;
+  }
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  int nparts = 0;
+  if (dynamic) {
+    const int64_t warps_per_block = kAmaxThreads / 32;
+    int64_t blocks = ceil_div(rows, warps_per_block);
+    if (blocks > static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM) blocks = static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM;
+    if (blocks > kMaxPartials) blocks = kMaxPartials;
+    if (blocks < 1) blocks = 1;
+    nparts = static_cast<int>(blocks);
+    amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
+                                                static_cast<float*>(workspace));
+    if (nvfp4_status e = launch_status()) return e;
+  }
+  QuantArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.rows = rows;
+  a.k = k;
+  a.ldx = ldx;
+  a.global_in = global_in;
+  a.partials = static_cast<const float*>(workspace);
+  a.nparts = nparts;
+  a.codes = codes;
+  a.sf = sf;
+  a.global_out = global_out;
+  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
+  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
+  const int64_t cap = static_cast<int64_t>(st->sms) * kQuantBlocksPerSM;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  quantize_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(a);
+  return launch_status();
+}
+
+size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+  (void)m;
+  (void)n;
+  (void)k;
+  return 0;
+}
+
+namespace {
+
+nvfp4_status encode_2d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base,
+                       uint64_t inner_bytes, uint64_t rows, uint32_t box_rows) {
+  cuuint64_t dims[2] = {inner_bytes, rows};
+  cuuint64_t strides[1] = {inner_bytes};
+  cuuint32_t box[2] = {128u, box_rows};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+// Scale factors as [row blocks][atoms][128 x uint32]: one box = whole atoms.
+nvfp4_status encode_sf(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base,
+                       int64_t rows, int64_t k, uint32_t box_row_blocks) {
+  const uint64_t n_ka = static_cast<uint64_t>(ceil_div(k, 64));
+  const uint64_t n_rb = static_cast<uint64_t>(ceil_div(rows, 128));
+  cuuint64_t dims[3] = {128u, n_ka, n_rb};
+  cuuint64_t strides[2] = {512u, n_ka * 512u};
+  cuuint32_t box[3] = {128u, 4u, box_row_blocks};
+  cuuint32_t estr[3] = {1u, 1u, 1u};
+  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT32, 3, const_cast<void*>(base), dims, strides,
+                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
+}  // namespace
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
+                        void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
+                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  using namespace nvfp4::gemm;
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!a_codes || !a_sf || !a_global || !b_codes || !b_sf || !b_global || !y)
+    return NVFP4_ERR_INVALID_ARG;
+  if (m < 1 || n < 1 || k < 1 || (y_dtype != 0 && y_dtype != 1) || ldy < n)
+    return NVFP4_ERR_INVALID_ARG;
+  if (k % 32 != 0 || m >= (int64_t{1} << 31) || n >= (int64_t{1} << 31) ||
+      k >= (int64_t{1} << 31))
+    return NVFP4_ERR_UNSUPPORTED;
+  const int64_t esize = y_dtype == 0 ? 2 : 4;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
+      !aligned(y, 16) || (ldy * esize) % 16 != 0 || !aligned(a_global, 4) || !aligned(b_global, 4))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (nvfp4_status e = get_encoder(&enc)) return e;
+
+  CUtensorMap tmA, tmB, tmSFA, tmSFB;
+  if (nvfp4_status e = encode_2d(enc, &tmA, a_codes, static_cast<uint64_t>(k / 2),
+                                 static_cast<uint64_t>(m), BM))
+    return e;
+  if (nvfp4_status e = encode_2d(enc, &tmB, b_codes, static_cast<uint64_t>(k / 2),
+                                 static_cast<uint64_t>(n), BN))
+    return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFA, a_sf, m, k, 1u)) return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFB, b_sf, n, k, 2u)) return e;
+
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!st->gemm_smem_set) {
+      if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(SMEM_BYTES)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+      }
+      st->gemm_smem_set = true;
+    }
+  }
+  Params p;
+  p.M = static_cast<int>(m);
+  p.N = static_cast<int>(n);
+  p.K = static_cast<int>(k);
+  p.num_m_blk = static_cast<int>(ceil_div(m, BM));
+  p.num_n_blk = static_cast<int>(ceil_div(n, BN));
+  p.num_k_tiles = static_cast<int>(ceil_div(k, BK));
+  p.a_global = a_global;
+  p.b_global = b_global;
+  p.y = y;
+  p.ldy = ldy;
+  p.y_fp32 = y_dtype;
+  const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
+  if (tiles >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;
+  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
+  gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
+      tmA, tmB, tmSFA, tmSFB, p);
+  return launch_status();
+}
+
+nvfp4_status nvfp4_fuse_group_scales(int n_modules, const int64_t* rows_per_module, int64_t k,
+                                     const uint8_t* const* sf_modules, const float* globals_in,
+                                     uint8_t* sf_fused, float* global_out,
+                                     nvfp4_stream_t stream) {
+  using namespace nvfp4::fold;
+  if (n_modules < 1 || n_modules > kMaxModules || !rows_per_module || !sf_modules ||
+      !globals_in || !sf_fused || !global_out || k <= 0)
+    return NVFP4_ERR_INVALID_ARG;
+  if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED;
+  FoldArgs a;
+  std::memset(&a, 0, sizeof a);
+  a.n = n_modules;
+  a.k = k;
+  a.n_ka = ceil_div(k, 64);
+  int64_t total = 0;
+  const uintptr_t out_lo = reinterpret_cast<uintptr_t>(sf_fused);
+  for (int i = 0; i < n_modules; ++i) {
+    if (rows_per_module[i] < 1 || sf_modules[i] == nullptr) return NVFP4_ERR_INVALID_ARG;
+    if (!aligned(sf_modules[i], 4)) return NVFP4_ERR_MISALIGNED;
+    a.row_start[i] = total;
+    a.sf_in[i] = sf_modules[i];
+    total += rows_per_module[i];
+  }
+  a.row_start[n_modules] = total;
+  a.total_rows = total;
+  const size_t out_bytes = nvfp4_sf_bytes(total, k);
+  const uintptr_t out_hi = out_lo + out_bytes;
+  for (int i = 0; i < n_modules; ++i) {
+    const uintptr_t lo = reinterpret_cast<uintptr_t>(sf_modules[i]);
+    const uintptr_t hi = lo + nvfp4_sf_bytes(rows_per_module[i], k);
+    if (lo < out_hi && out_lo < hi) return NVFP4_ERR_INVALID_ARG;  // in place is not allowed
+  }
+  const uintptr_t g_lo = reinterpret_cast<uintptr_t>(globals_in);
+  const uintptr_t g_out = reinterpret_cast<uintptr_t>(global_out);
+  if (g_out + sizeof(float) > g_lo && g_out < g_lo + sizeof(float) * n_modules)
+    return NVFP4_ERR_INVALID_ARG;  // g* must not overwrite an input global mid-kernel
+  if (!aligned(sf_fused, 16) || !aligned(globals_in, 4) || !aligned(global_out, 4))
+    return NVFP4_ERR_MISALIGNED;
+  a.g_in = globals_in;
+  a.sf_out = sf_fused;
+  a.g_out = global_out;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  const int64_t words = static_cast<int64_t>(out_bytes / 4);
+  int64_t blocks = ceil_div(words, kThreads);
+  if (blocks > static_cast<int64_t>(st->sms) * 8) blocks = static_cast<int64_t>(st->sms) * 8;
+  if (blocks < 1) blocks = 1;
+  fold_kernel<<<static_cast<unsigned>(blocks), kThreads, 0,
+                reinterpret_cast<cudaStream_t>(stream)>>>(a);
+  return launch_status();
+}
+
+nvfp4_status nvfp4_silu_mul(const void* y, int64_t m, int64_t n, int64_t ldy, void* h,
+                            int64_t ldh, nvfp4_stream_t stream) {
+  using namespace nvfp4::act;
+  if (!y || !h || m < 0 || n < 1 || ldy < 2 * n || ldh < n) return NVFP4_ERR_INVALID_ARG;
+  if (n % 8 != 0) return NVFP4_ERR_UNSUPPORTED;
+  if (ldy % 8 != 0 || ldh % 8 != 0 || !aligned(y, 16) || !aligned(h, 16))
+    return NVFP4_ERR_MISALIGNED;
+  if (m == 0) return NVFP4_OK;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  int64_t blocks = ceil_div(m, kThreads / 32);
+  if (blocks > static_cast<int64_t>(st->sms) * 8) blocks = static_cast<int64_t>(st->sms) * 8;
+  silu_mul_kernel<<<static_cast<unsigned>(blocks), kThreads, 0,
+                    reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<const uint16_t*>(y), m, n, ldy, static_cast<uint16_t*>(h), ldh);
+  return launch_status();
+}
+
+nvfp4_status nvfp4_read_fault(nvfp4_stream_t stream, uint32_t* fault_out) {
+  if (fault_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  unsigned int v = 0;
+  const unsigned int zero = 0;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess ||
+      cudaMemcpyFromSymbol(&v, nvfp4::g_fault_word, sizeof v) != cudaSuccess ||
+      cudaMemcpyToSymbol(nvfp4::g_fault_word, &zero, sizeof zero) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  *fault_out = v;
+  return v ? NVFP4_ERR_TIMEOUT : NVFP4_OK;
+}
+
+}  // extern "C"

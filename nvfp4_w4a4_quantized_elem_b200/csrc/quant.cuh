@@ -1,0 +1,199 @@
+// quant.cuh — NVFP4 quantization of a bf16 tensor (weights or activations).
+//
+// Format: news article "Qwen3.8-27B最激进4bit量化开源，权重显存暴降2.9倍！" §02
+// (NVFP4 量化格式): E2M1 values, one E4M3 scale per 16 contiguous elements,
+// one FP32 global scale per tensor; W4A4 applies it to activations on the fly.
+// Convention (FP32, round-to-nearest-even at every step):
+//   g = 2688 / amax;  s = E4M3(amax_b / 6 * g);  code = E2M1(x * (g / dec(s))).
+//
+// Two kernels:
+//   amax_kernel      one pass over x, one partial max per CTA (no atomics, so
+//                    the workspace needs no initialisation);
+//   quantize_kernel  every CTA first reduces the partials to g (a few hundred
+//                    floats from L2), then quantizes. A warp task is one
+//                    (128-row block, row l in 0..31, 4 consecutive 64-column
+//                    atoms): the warp reads rows l, l+32, l+64, l+96 — four
+//                    full 128-byte lines per atom — so each lane holds 8
+//                    elements (half a 16-element block) and the 4 row groups
+//                    x 4 blocks of scales form one whole 16-byte line of the
+//                    swizzled scale atom, written with a single store.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace nvfp4 {
+namespace quant {
+
+constexpr int kAmaxThreads = 1024;
+constexpr int kAmaxBlocksPerSM = 2;
+constexpr int kMaxPartials = 4096;            // workspace = 16 KiB
+constexpr int kQuantThreads = 256;
+constexpr int kQuantBlocksPerSM = 8;
+constexpr int kAtomsPerTask = 4;
+
+__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// max |x| of 8 bf16 values, as the 15-bit magnitude pattern (sign cleared);
+// for non-negative floats the bit pattern orders like the value.
+__device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
+  const uint32_t m = 0x7FFF7FFFu;
+  const uint32_t w = __vmaxu2(__vmaxu2(v.x & m, v.y & m), __vmaxu2(v.z & m, v.w & m));
+  return max(w & 0xFFFFu, w >> 16);
+}
+
+__global__ void __launch_bounds__(kAmaxThreads)
+    amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ldx,
+                float* __restrict__ partials) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const int64_t chunks = k >> 3;  // 16-byte chunks per row
+  uint32_t m = 0;
+  for (int64_t r = warp; r < rows; r += nwarps) {
+    const uint16_t* row = x + r * ldx;
+    int64_t c = lane;
+    for (; c + 96 < chunks; c += 128) {
+      const uint4 v0 = ldg_stream(row + c * 8);
+      const uint4 v1 = ldg_stream(row + (c + 32) * 8);
+      const uint4 v2 = ldg_stream(row + (c + 64) * 8);
+      const uint4 v3 = ldg_stream(row + (c + 96) * 8);
+      m = max(m, max(max(absmax_bits8(v0), absmax_bits8(v1)),
+                     max(absmax_bits8(v2), absmax_bits8(v3))));
+    }
+    for (; c < chunks; c += 32) m = max(m, absmax_bits8(ldg_stream(row + c * 8)));
+  }
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  __shared__ uint32_t s_red[32];
+  if (lane == 0) s_red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    uint32_t v = threadIdx.x < (blockDim.x >> 5) ? s_red[threadIdx.x] : 0u;
+    v = __reduce_max_sync(0xFFFFFFFFu, v);
+    if (threadIdx.x == 0) partials[blockIdx.x] = __uint_as_float(v << 16);
+  }
+}
+
+struct QuantArgs {
+  const uint16_t* x;
+  int64_t rows, k, ldx;
+  const float* global_in;   // static mode when non-null
+  const float* partials;    // dynamic mode: per-CTA maxima of amax_kernel
+  int nparts;
+  uint8_t* codes;
+  uint8_t* sf;
+  float* global_out;
+};
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs a) {
+  __shared__ float s_g;
+  __shared__ uint32_t s_red[kQuantThreads / 32];
+  const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+
+  // ---- global scale g (identical in every CTA) -----------------------------
+  if (a.global_in != nullptr) {
+    if (threadIdx.x == 0) s_g = *a.global_in;
+  } else {
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < a.nparts; i += blockDim.x)
+      m = max(m, __float_as_uint(a.partials[i]));  // non-negative: bits order as values
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) s_red[wib] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t mm = 0;
+      for (int w = 0; w < kQuantThreads / 32; ++w) mm = max(mm, s_red[w]);
+      const float amax = __uint_as_float(mm);
+      float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, amax);
+      if (!isfinite(g)) g = 1.0f;
+      s_g = g;
+    }
+  }
+  __syncthreads();
+  const float g = s_g;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *a.global_out = g;
+
+  // ---- blocks ----------------------------------------------------------------
+  const int64_t n_rb = (a.rows + 127) / 128;
+  const int64_t n_ka = (a.k + 63) / 64;  // 512-byte atoms per 128-row block
+  const int64_t n_kc = (n_ka + kAtomsPerTask - 1) / kAtomsPerTask;
+  const int64_t n_tasks = n_rb * 32 * n_kc;
+  const int grp = lane >> 3;  // row group: row l + 32*grp
+  const int j = lane & 7;     // 16-byte chunk of the row's 128-byte atom slice
+  const int64_t half_k = a.k >> 1;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+
+  for (int64_t t = warp; t < n_tasks; t += nwarps) {
+    const int64_t kc = t % n_kc;
+    const int64_t tl = t / n_kc;
+    const int l = static_cast<int>(tl & 31);
+    const int64_t rb = tl >> 5;
+    const int64_t row = rb * 128 + grp * 32 + l;
+    const bool row_ok = row < a.rows;
+    const uint16_t* xrow = a.x + row * a.ldx;
+
+    uint4 v[kAtomsPerTask];
+#pragma unroll
+    for (int u = 0; u < kAtomsPerTask; ++u) {
+      const int64_t col = (kc * kAtomsPerTask + u) * 64 + j * 8;
+      v[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (row_ok && col < a.k) v[u] = ldg_stream(xrow + col);
+    }
+#pragma unroll
+    for (int u = 0; u < kAtomsPerTask; ++u) {
+      const int64_t ka = kc * kAtomsPerTask + u;
+      if (ka >= n_ka) break;  // warp-uniform
+      const int64_t col = ka * 64 + j * 8;
+      const bool ok = row_ok && col < a.k;
+
+      // block amax: this lane's 8 elements and its partner lane's 8
+      uint32_t mb = absmax_bits8(v[u]);
+      mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
+      const float amax_b = __uint_as_float(mb << 16);
+      const float t6 = __fdiv_rn(amax_b, 6.0f);
+      const uint32_t s = ptx::cvt_e4m3(__fmul_rn(t6, g));
+      const float ds = ptx::e4m3_value(s);
+      const float r = (ds == 0.0f) ? 0.0f : __fdiv_rn(g, ds);  // r = 0 keeps only signs
+
+      float f[8];
+      f[0] = __fmul_rn(bf16_lo(v[u].x), r);
+      f[1] = __fmul_rn(bf16_hi(v[u].x), r);
+      f[2] = __fmul_rn(bf16_lo(v[u].y), r);
+      f[3] = __fmul_rn(bf16_hi(v[u].y), r);
+      f[4] = __fmul_rn(bf16_lo(v[u].z), r);
+      f[5] = __fmul_rn(bf16_hi(v[u].z), r);
+      f[6] = __fmul_rn(bf16_lo(v[u].w), r);
+      f[7] = __fmul_rn(bf16_hi(v[u].w), r);
+      const uint32_t packed = ptx::cvt_e2m1x8(f);
+      if (ok) *reinterpret_cast<uint32_t*>(a.codes + row * half_k + (col >> 1)) = packed;
+
+      // scales: lanes 8g+{0,2,4,6} hold blocks 0..3 of row group g
+      const int base = grp * 8;
+      const uint32_t b0 = __shfl_sync(0xFFFFFFFFu, s, base + 0);
+      const uint32_t b1 = __shfl_sync(0xFFFFFFFFu, s, base + 2);
+      const uint32_t b2 = __shfl_sync(0xFFFFFFFFu, s, base + 4);
+      const uint32_t b3 = __shfl_sync(0xFFFFFFFFu, s, base + 6);
+      const uint32_t word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+      const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, word, 0);
+      const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, word, 8);
+      const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, word, 16);
+      const uint32_t w3 = __shfl_sync(0xFFFFFFFFu, word, 24);
+      if (lane == 0)
+        *reinterpret_cast<uint4*>(a.sf + (rb * n_ka + ka) * 512 + l * 16) =
+            make_uint4(w0, w1, w2, w3);
+    }
+  }
+}
+
+}  // namespace quant
+}  // namespace nvfp4

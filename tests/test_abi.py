@@ -1,0 +1,121 @@
+"""The C-ABI library loads, exports every symbol include/nvfp4.h declares, and
+rejects bad arguments on the host (no GPU needed: argument checks return a
+status before anything touches CUDA)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4.h")
+
+OK, INVALID, UNSUPPORTED, MISALIGNED = 0, 1, 2, 3
+
+
+@pytest.fixture(scope="module")
+def L():
+    from nvfp4_w4a4_quantized_elem_b200 import build, nvfp4
+    build.build()
+    return nvfp4.lib()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvfp4_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for f in ("nvfp4_quantize", "nvfp4_gemm", "nvfp4_fuse_group_scales"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    from nvfp4_w4a4_quantized_elem_b200 import nvfp4
+    names = declared_functions()
+    assert sorted(nvfp4.EXPORTS) == names
+    for name in names:
+        assert hasattr(L, name), name
+
+
+def test_status_strings(L):
+    for code, name in [(0, b"NVFP4_OK"), (1, b"NVFP4_ERR_INVALID_ARG"), (5, b"NVFP4_ERR_TIMEOUT")]:
+        assert L.nvfp4_status_string(code) == name
+
+
+def test_sf_bytes(L):
+    assert L.nvfp4_sf_bytes(64, 256) == 128 * 16
+    assert L.nvfp4_sf_bytes(12384, 5120) == 12416 * 320
+    assert L.nvfp4_sf_bytes(1, 16) == 128 * 4
+    assert L.nvfp4_sf_bytes(0, 16) == 0
+    assert L.nvfp4_sf_bytes(4, 24) == 0     # k % 16 != 0
+    assert L.nvfp4_sf_bytes(-1, 16) == 0
+
+
+def test_sf_bytes_matches_oracle(L, orc):
+    for rows, k in [(1, 16), (130, 80), (8192, 5120), (48, 5120), (32768, 17408)]:
+        assert L.nvfp4_sf_bytes(rows, k) == orc.sf_bytes(rows, k)
+
+
+P = ctypes.c_void_p
+FAKE = 1 << 20  # an aligned, never-dereferenced address (checks fail first)
+
+
+def q(L, x=FAKE, rows=4, k=32, ldx=32, gin=None, codes=FAKE, sf=FAKE, gout=FAKE,
+      ws=FAKE, wsb=1 << 16):
+    return L.nvfp4_quantize(P(x), rows, k, ldx, P(gin), P(codes), P(sf), P(gout), P(ws), wsb, None)
+
+
+def test_quantize_argument_checks(L):
+    assert q(L, k=24) == UNSUPPORTED
+    assert q(L, k=0) == INVALID
+    assert q(L, rows=-1) == INVALID
+    assert q(L, x=None) == INVALID
+    assert q(L, gout=None) == INVALID
+    assert q(L, ldx=16) == INVALID           # ldx < k
+    assert q(L, ldx=36) == MISALIGNED        # ldx % 8
+    assert q(L, x=FAKE + 8) == MISALIGNED
+    assert q(L, sf=FAKE + 4) == MISALIGNED
+    assert q(L, codes=FAKE + 2) == MISALIGNED
+    assert q(L, ws=None) == INVALID          # dynamic mode needs workspace
+    assert q(L, wsb=16) == INVALID
+
+
+def g(L, a=FAKE, asf=FAKE, ag=FAKE, b=FAKE, bsf=FAKE, bg=FAKE, y=FAKE, yd=0, ldy=64,
+      m=8, n=64, k=64):
+    return L.nvfp4_gemm(P(a), P(asf), P(ag), P(b), P(bsf), P(bg), P(y), yd, ldy, m, n, k,
+                        None, 0, None)
+
+
+def test_gemm_argument_checks(L):
+    assert g(L, k=48) == UNSUPPORTED         # k % 32
+    assert g(L, m=0) == INVALID
+    assert g(L, yd=2) == INVALID
+    assert g(L, ldy=32) == INVALID           # ldy < n
+    assert g(L, n=60, ldy=60) == MISALIGNED  # 120-byte row pitch
+    assert g(L, a=FAKE + 8) == MISALIGNED
+    assert g(L, bsf=FAKE + 4) == MISALIGNED
+    assert g(L, ag=None) == INVALID
+
+
+def test_fuse_argument_checks(L):
+    rows = (ctypes.c_int64 * 2)(48, 48)
+    ptrs = (ctypes.c_void_p * 2)(FAKE, FAKE + (1 << 16))
+    f = L.nvfp4_fuse_group_scales
+    cast = lambda a: ctypes.cast(a, P)
+    assert f(0, cast(rows), 64, cast(ptrs), P(FAKE), P(FAKE * 4), P(FAKE * 8), None) == INVALID
+    assert f(17, cast(rows), 64, cast(ptrs), P(FAKE), P(FAKE * 4), P(FAKE * 8), None) == INVALID
+    assert f(2, cast(rows), 40, cast(ptrs), P(FAKE), P(FAKE * 4), P(FAKE * 8), None) == UNSUPPORTED
+    # output overlapping an input scale buffer (in place) is refused
+    assert f(2, cast(rows), 64, cast(ptrs), P(FAKE * 2), P(FAKE), P(FAKE * 8), None) == INVALID
+    # g* written over one of the input globals is refused
+    assert f(2, cast(rows), 64, cast(ptrs), P(FAKE * 2), P(FAKE * 4), P(FAKE * 2 + 4), None) == INVALID
+
+
+def test_silu_argument_checks(L):
+    f = L.nvfp4_silu_mul
+    assert f(P(FAKE), 4, 12, 24, P(FAKE), 16, None) == UNSUPPORTED  # n % 8
+    assert f(P(FAKE), 4, 16, 16, P(FAKE), 16, None) == INVALID      # ldy < 2n
+    assert f(P(FAKE + 2), 4, 16, 32, P(FAKE), 16, None) == MISALIGNED

@@ -1,0 +1,94 @@
+"""GPU parity of nvfp4_gemm against the FP64 oracle GEMM of the dequantized
+operands (news article "Qwen3.8-27B最激进4bit量化开源…" §02: W4A4 GEMM on the
+4-bit tensor cores). Operands are quantized by the oracle and uploaded, so a
+GEMM failure cannot hide behind a quantizer failure. Tolerance: parity.py.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity import assert_quant_equal, bits, gemm_check, norms, upload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    from nvfp4_w4a4_quantized_elem_b200 import build, nvfp4
+    build.build()
+    return nvfp4
+
+
+def gaussian(rows, k, seed, sigma=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn((rows, k), generator=g) * sigma).to(torch.bfloat16)
+
+
+def run_case(nv, orc, x, w, dtypes=(torch.bfloat16, torch.float32), what=""):
+    qa, qb = orc.quantize(bits(x)), orc.quantize(bits(w))
+    ref = orc.gemm(qa, qb)
+    rn, cn = norms(orc, qa), norms(orc, qb)
+    A, B = upload(qa), upload(qb)
+    for dt in dtypes:
+        y = nv.gemm(A, B, out_dtype=dt)
+        torch.cuda.synchronize()
+        gemm_check(y, ref, rn, cn, f"{what} {dt}")
+    assert nv.read_fault() == 0
+
+
+def test_gemm_tiny(nv, orc):
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+    cfg = wl.tiny()
+    run_case(nv, orc, cfg.x(), cfg.w(), what="tiny")
+
+
+@pytest.mark.parametrize("m,n,k", [(1, 8, 32), (7, 48, 64), (130, 136, 96), (128, 256, 256),
+                                   (300, 520, 288), (129, 257, 1024), (256, 512, 5120),
+                                   (513, 1000, 2080)])
+def test_gemm_ragged(nv, orc, m, n, k):
+    run_case(nv, orc, gaussian(m, k, m + k), gaussian(n, k, n + 2 * k, 0.02), what=f"{m}x{n}x{k}")
+
+
+def test_gemm_output_pitch(nv, orc):
+    x, w = gaussian(100, 256, 1), gaussian(200, 256, 2, 0.02)
+    qa, qb = orc.quantize(bits(x)), orc.quantize(bits(w))
+    ref = orc.gemm(qa, qb)
+    big = torch.full((100, 264), 7.0, dtype=torch.bfloat16, device="cuda")
+    y = nv.gemm(upload(qa), upload(qb), out=big[:, :200])
+    torch.cuda.synchronize()
+    gemm_check(y, ref, norms(orc, qa), norms(orc, qb), "pitched")
+    assert torch.all(big[:, 200:] == 7.0)  # nothing written past n
+
+
+def test_gemm_zero_scales_and_extremes(nv, orc):
+    # rows spanning 40 binades (subnormal and zero block scales) and all-zero rows
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal((256, 512)) * np.exp2(rng.uniform(-30, 8, (256, 1)))).astype(np.float32)
+    x[10] = 0.0
+    w = (rng.standard_normal((384, 512)) * 0.02).astype(np.float32)
+    run_case(nv, orc, torch.from_numpy(x).to(torch.bfloat16),
+             torch.from_numpy(w).to(torch.bfloat16), what="extremes")
+
+
+def test_gemm_outlier_config_full(nv, orc):
+    """X 8192x5120 (8 outlier channels x50) @ W 5120x5120: GPU quantizes X and
+    W (checked bit-exact), GPU GEMM vs the full FP64 oracle GEMM."""
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+    cfg = wl.outlier()
+    x, w = cfg.x(), cfg.w()
+    A, B = nv.quantize(x.cuda()), nv.quantize(w.cuda())
+    qa, qb = orc.quantize(bits(x)), orc.quantize(bits(w))
+    assert_quant_equal(A, qa, "X")
+    assert_quant_equal(B, qb, "W")
+    y = nv.gemm(A, B)
+    torch.cuda.synchronize()
+    ref = orc.gemm(qa, qb)
+    gemm_check(y, ref, norms(orc, qa), norms(orc, qb), "outlier full")
+
+
+@pytest.mark.parametrize("m", [1, 8, 32, 128, 256])
+@pytest.mark.parametrize("k,n", [(5120, 17408), (17408, 5120)])
+def test_gemm_decode_shapes(nv, orc, m, k, n):
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+    cfg = wl.decode(m, k, n)
+    run_case(nv, orc, cfg.x(), cfg.w(), dtypes=(torch.bfloat16,), what=cfg.name)
