@@ -29,8 +29,12 @@ def run_case(nv, orc, x, w, dtypes=(torch.bfloat16, torch.float32), what=""):
     ref = orc.gemm(qa, qb)
     rn, cn = norms(orc, qa), norms(orc, qb)
     A, B = upload(qa), upload(qb)
+    m, n = qa.rows, qb.rows
     for dt in dtypes:
-        y = nv.gemm(A, B, out_dtype=dt)
+        # the output row pitch must be a multiple of 16 bytes: pad it
+        per16 = 16 // torch.tensor([], dtype=dt).element_size()
+        ld = -(-n // per16) * per16
+        y = nv.gemm(A, B, out=torch.empty((m, ld), dtype=dt, device="cuda")[:, :n])
         torch.cuda.synchronize()
         gemm_check(y, ref, rn, cn, f"{what} {dt}")
     assert nv.read_fault() == 0
