@@ -127,6 +127,28 @@ class ClockSampler:
                 "samples": len(sm), "window": window}
 
 
+# ------------------------------------------------------------- multi-rank --
+
+def rank_x_seed(rank: int) -> int:
+    """Each replica quantizes its own batch: per-rank activation seed."""
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+    return wl.SEED_X + 1000 * rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """Device time of the job = the slowest rank (MAX all-reduce)."""
+    if dist is None:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job TFLOP/s: every rank's FLOPs over the slowest rank's time."""
+    return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # --------------------------------------------------------------- workloads --
 
 def make_workload(name: str, rank: int):
@@ -134,7 +156,7 @@ def make_workload(name: str, rank: int):
     from nvfp4_w4a4_quantized_elem_b200 import nvfp4, workloads as wl
     if name == "outlier":
         cfg = wl.outlier()
-        cfg.x_seed = wl.SEED_X + 1000 * rank
+        cfg.x_seed = rank_x_seed(rank)
         x = cfg.x().cuda()
         W = nvfp4.quantize(cfg.w().cuda())
         gemms = [(cfg.m, cfg.n, cfg.k)]
@@ -143,7 +165,7 @@ def make_workload(name: str, rank: int):
         return dict(x=x, W=W, gemms=gemms, desc=desc, kind="linear", m=cfg.m, n=cfg.n, k=cfg.k)
     if name == "gdn_fused":
         cfg = wl.gdn_fused()
-        x = wl.gaussian_bf16(cfg.m, cfg.k, 1.0, wl.SEED_X + 1000 * rank).cuda()
+        x = wl.gaussian_bf16(cfg.m, cfg.k, 1.0, rank_x_seed(rank)).cuda()
         mods = [nvfp4.quantize(w.cuda()) for w in cfg.weights()]
         W = nvfp4.fuse_group(mods)
         desc = (f"gdn_fused: X {cfg.m}x{cfg.k} @ fused qkv|z|a|b {cfg.n}x{cfg.k} "
@@ -290,13 +312,9 @@ def run_gpu(args):
     step_ms = [events[i][0].elapsed_time(events[i][nph - 1]) for i in range(args.steps)]
     quant_ms = [events[i][0].elapsed_time(events[i][1]) for i in range(args.steps)]
     gemm_ms = [events[i][1].elapsed_time(events[i][2]) for i in range(args.steps)]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / args.steps
-    value = flops * world / (ms_per_step * 1e-3) / 1e12
+    value = job_throughput(flops, world, ms_per_step)
 
     # component figures on this rank
     m, k = wk["x"].shape
@@ -325,11 +343,8 @@ def run_gpu(args):
     amax_gbs = elems * AMAX_BYTES_PER_ELEM / (amax_ms * 1e-3) / 1e9
 
     e2e = measure_e2e(step, wk, stream, flops, args)
-    if dist is not None:
-        t = torch.tensor([e2e["ms_per_step"]], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e["ms_per_step"] = float(t.item())
-        e2e["value"] = flops * world / (e2e["ms_per_step"] * 1e-3) / 1e12
+    e2e["ms_per_step"] = max_over_ranks(e2e["ms_per_step"], dist, "cuda")
+    e2e["value"] = job_throughput(flops, world, e2e["ms_per_step"])
 
     assert nvfp4.read_fault(stream) == 0
     traffic = dram_traffic(args.workload)
