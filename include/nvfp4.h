@@ -106,6 +106,40 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
                             float* global_out, void* workspace,
                             size_t workspace_bytes, nvfp4_stream_t stream);
 
+/*
+ * nvfp4_quantize_noalloc — nvfp4_quantize for callers that cannot allocate
+ * device memory. The paper has no counterpart of this entry point; it exists
+ * for integration only. Some callers are handed nothing but their input and
+ * output buffers and may not call cudaMalloc themselves: a plugin running
+ * inside another framework whose allocator owns all device memory, or a
+ * runtime that forbids cudaMalloc after start-up because the call can
+ * synchronise the whole device and break its latency budget. This variant
+ * takes no workspace: the per-CTA partial maxima of the amax pass live in a
+ * file-scope device array of NVFP4_NOALLOC_MAX_PARTIALS floats (4 KiB) that
+ * every GPU which loads the library holds until the process exits.
+ *
+ * Arguments, layouts, results and errors are those of nvfp4_quantize (minus
+ * the workspace pair). Additionally:
+ *   - NVFP4_ERR_UNSUPPORTED if the amax pass would need more than
+ *     NVFP4_NOALLOC_MAX_PARTIALS CTAs (it launches min(ceil(rows/32),
+ *     2 x SM count) of them; 296 on a 148-SM B200).
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before any stream capture. Later calls allocate nothing and call no
+ *     allocating routine.
+ *   - Every call on a device shares the one array and it keeps the last
+ *     call's contents. Nothing in it needs to start at zero: each slot the
+ *     quantizer reads is first written by the same call's amax pass. Calls
+ *     whose kernels overlap on the GPU (e.g. on two concurrently running
+ *     streams of one device) race on the array and may produce wrong scales;
+ *     serialise them.
+ */
+#define NVFP4_NOALLOC_MAX_PARTIALS 1024
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k,
+                                    int64_t ldx, const float* global_in,
+                                    uint8_t* codes, uint8_t* sf,
+                                    float* global_out, nvfp4_stream_t stream);
+
 /* Workspace bytes nvfp4_gemm needs (0 for every shape the current kernels
  * handle; kept so callers need not change when split-K arrives). */
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);

@@ -26,6 +26,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
   int sms = 0;
   bool gemm_smem_set = false;
+  float* noalloc_partials = nullptr;  // device address of g_noalloc_partials
 };
 
 std::mutex g_mutex;
@@ -76,6 +77,26 @@ nvfp4_status launch_status() {
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Scratch of nvfp4_quantize_noalloc: the amax pass's per-CTA partial maxima.
+// Host code must not use this name as a pointer (it is a host-side stand-in);
+// the device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) float g_noalloc_partials[NVFP4_NOALLOC_MAX_PARTIALS];
+
+// First call on the current device: look up the array's device address.
+nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (st->noalloc_partials == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_partials) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    st->noalloc_partials = static_cast<float*>(p);
+  }
+  *out = st->noalloc_partials;
+  return NVFP4_OK;
+}
 
 }  // namespace
 
@@ -146,6 +167,56 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
   a.ldx = ldx;
   a.global_in = global_in;
   a.partials = static_cast<const float*>(workspace);
+  a.nparts = nparts;
+  a.codes = codes;
+  a.sf = sf;
+  a.global_out = global_out;
+  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
+  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
+  const int64_t cap = static_cast<int64_t>(st->sms) * kQuantBlocksPerSM;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  quantize_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(a);
+  return launch_status();
+}
+
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k, int64_t ldx,
+                                    const float* global_in, uint8_t* codes, uint8_t* sf,
+                                    float* global_out, nvfp4_stream_t stream) {
+  using namespace nvfp4::quant;
+  if (rows < 0 || k <= 0 || global_out == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED;
+  if (rows > 0 && (x == nullptr || codes == nullptr || sf == nullptr)) return NVFP4_ERR_INVALID_ARG;
+  if (ldx < k) return NVFP4_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(codes, 4) || !aligned(sf, 16) ||
+      !aligned(global_out, 4))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  float* partials = nullptr;
+  if (nvfp4_status e = noalloc_scratch(st, &partials)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  int nparts = 0;
+  if (global_in == nullptr) {
+    int64_t blocks = ceil_div(rows, kAmaxThreads / 32);
+    if (blocks > static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM)
+      blocks = static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM;
+    if (blocks < 1) blocks = 1;
+    if (blocks > NVFP4_NOALLOC_MAX_PARTIALS) return NVFP4_ERR_UNSUPPORTED;
+    nparts = static_cast<int>(blocks);
+    amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
+                                                partials);
+    if (nvfp4_status e = launch_status()) return e;
+  }
+  QuantArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.rows = rows;
+  a.k = k;
+  a.ldx = ldx;
+  a.global_in = global_in;
+  a.partials = partials;
   a.nparts = nparts;
   a.codes = codes;
   a.sf = sf;

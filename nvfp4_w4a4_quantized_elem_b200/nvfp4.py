@@ -24,7 +24,7 @@ STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPO
 
 # every symbol include/nvfp4.h declares
 EXPORTS = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_quantize_workspace_bytes",
-           "nvfp4_quantize", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm",
+           "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm",
            "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault")
 
 _lib = None
@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_sf_bytes": (SZ, [I64, I64]),
             "nvfp4_quantize_workspace_bytes": (SZ, [I64, I64]),
             "nvfp4_quantize": (I, [P, I64, I64, I64, P, P, P, P, P, SZ, P]),
+            "nvfp4_quantize_noalloc": (I, [P, I64, I64, I64, P, P, P, P, P]),
             "nvfp4_gemm_workspace_bytes": (SZ, [I64, I64, I64]),
             "nvfp4_gemm": (I, [P, P, P, P, P, P, P, I, I64, I64, I64, I64, P, SZ, P]),
             "nvfp4_fuse_group_scales": (I, [I, P, I64, P, P, P, P, P]),
@@ -134,6 +135,23 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None,
                               _ptr(out.codes), _ptr(out.sf), _ptr(out.global_scale),
                               _ptr(workspace), ws_bytes, _stream(stream))
     _check(st, "nvfp4_quantize")
+    return out
+
+
+def quantize_noalloc(x: torch.Tensor, out: NVFP4Tensor, global_scale: torch.Tensor | None = None,
+                     stream: torch.cuda.Stream | None = None) -> NVFP4Tensor:
+    """nvfp4_quantize_noalloc: as quantize(), for callers that cannot
+    allocate device memory. No workspace: the amax pass uses a fixed device
+    array inside the library (shared by every call on the device; calls that
+    overlap on the GPU race). The caller supplies the output buffers."""
+    _require_cuda(x, "x", torch.bfloat16)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit stride along k")
+    rows, k = x.shape
+    st = lib().nvfp4_quantize_noalloc(_ptr(x), rows, k, x.stride(0), _ptr(global_scale),
+                                      _ptr(out.codes), _ptr(out.sf), _ptr(out.global_scale),
+                                      _stream(stream))
+    _check(st, "nvfp4_quantize_noalloc")
     return out
 
 
