@@ -7,21 +7,34 @@
 // tensor cores; the per-16 E4M3 scales are applied inside the MMA and the two
 // FP32 globals in the epilogue.
 //
-// Design (one CTA per SM, persistent over 128x256 output tiles):
-//   warp 0  TMA producer: A (128 rows x 128 B), B (256 x 128 B) with 128-byte
-//           swizzle, and the two scale tiles (whole 512-byte atoms) into a
-//           4-stage shared-memory ring guarded by full/empty mbarriers;
-//   warp 1  allocates 512 tensor-memory columns; one thread copies each
-//           stage's scale atoms into tensor memory (tcgen05.cp 32x128b.warpx4)
-//           and issues 4 x tcgen05.mma.kind::mxf4nvf4.block16 (K = 64 each)
-//           per 256-element k-tile into a 128x256 FP32 accumulator;
-//   warps 2..9  epilogue: two warps per tensor-memory lane quarter, each
-//           drains 128 accumulator columns into registers, releases the
-//           accumulator (so the next tile's MMAs start at once), then scales
-//           by 1/(g_a g_b), converts and stores its row.
+// Design: persistent CTA pairs (clusters of 2, one CTA per SM) over 256x256
+// output tiles. The pair issues one M = 256 MMA (tcgen05 cta_group::2): the
+// even CTA's tensor memory accumulates tile rows 0-127, the odd CTA's rows
+// 128-255, and each CTA stages only its own half of A and half of B, so a
+// stage costs each SM 38 KiB of shared memory instead of 54 KiB for a 1-SM
+// 128x256 tile.
+//   warp 0  TMA producer (both CTAs): A (128 rows x 128 B) and B (128 N rows x
+//           128 B) with 128-byte swizzle, this CTA's A scale atoms and all 256
+//           B-row scale atoms, into a 5-stage ring. Both CTAs' copies signal
+//           the even CTA's full barrier, which expects the pair's bytes.
+//   warp 1  allocates 512 tensor-memory columns in both CTAs; in the even CTA
+//           one thread issues 4 MMAs (kind::mxf4nvf4.block16, K = 64) per
+//           256-element k-tile, then commits to the empty barrier of both
+//           CTAs and to the scale buffer's empty barrier.
+//   warps 2, 3  (even CTA) copy each stage's scale atoms into one of 4
+//           tensor-memory scale buffers (tcgen05.cp 32x128b.warpx4, both
+//           CTAs), 6 of the 12 copies each, and commit to that buffer's full
+//           barrier. Each tcgen05.cp costs a fixed ~50 cycles whatever its
+//           size; issued from the MMA thread the 12 copies per k-tile
+//           serialise with the 4 MMAs (about half the tensor-pipe time), and
+//           one copy warp alone issues slower than the MMAs consume.
+//   warps 4..11  epilogue (both CTAs): two warps per tensor-memory lane
+//           quarter drain 128 columns each into registers, release the
+//           accumulator (arrive on the even CTA's barrier), then scale by
+//           1/(g_a g_b), convert and store.
 // Every mbarrier wait is bounded in time; on expiry the kernel records a fault
-// word, every role stops, in-flight copies and MMAs are drained (again with a
-// bound) and tensor memory is released before the CTA exits.
+// word, both CTAs of the pair stop, in-flight copies and MMAs are drained
+// (again with a bound) and tensor memory is released before the CTAs exit.
 #pragma once
 
 #include <cuda.h>
@@ -37,34 +50,39 @@ __device__ unsigned int g_fault_word;
 
 namespace gemm {
 
-constexpr int BM = 128;
+constexpr int BM = 256;                       // tile rows (128 per CTA of the pair)
 constexpr int BN = 256;
 constexpr int BK = 256;                       // FP4 elements per k-tile
 constexpr int BK_BYTES = BK / 2;              // 128 bytes: one swizzle row
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK_BYTES;        // 16 KiB
-constexpr int B_BYTES = BN * BK_BYTES;        // 32 KiB
-constexpr int SFA_BYTES = BM * (BK / 16);     // 2 KiB = 4 atoms
+constexpr int HALF = 128;                     // rows of A / B per CTA
+constexpr int STAGES = 5;
+constexpr int A_BYTES = HALF * BK_BYTES;      // 16 KiB
+constexpr int B_BYTES = HALF * BK_BYTES;      // 16 KiB
+constexpr int SFA_BYTES = HALF * (BK / 16);   // 2 KiB = 4 atoms (this CTA's rows)
 constexpr int SFB_BYTES = BN * (BK / 16);     // 4 KiB = 2 row blocks x 4 atoms
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
 constexpr int NUM_EPI_WARPS = 8;
-constexpr int NUM_THREADS = 64 + 32 * NUM_EPI_WARPS;
+constexpr int SF_WARP0 = 2;                   // warps 2, 3: scale copies
+constexpr int NUM_SF_WARPS = 2;
+constexpr int EPI_WARP0 = SF_WARP0 + NUM_SF_WARPS;  // warps 4..11
+constexpr int NUM_THREADS = 32 * EPI_WARP0 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;               // [0, 256): FP32 accumulator
-constexpr uint32_t SFA_COL = 256;             // 2 buffers x 16 columns
-constexpr uint32_t SFB_COL = 288;             // 2 buffers x 32 columns
-constexpr int GROUP_M = 8;                    // tile raster: 8 M-blocks per band
-constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 256;
+constexpr int NSF = 4;                        // tensor-memory scale buffers
+constexpr uint32_t SF_COL = 256;              // NSF x 48 columns: [A 16 | B 32]
+constexpr uint32_t SF_BUF_COLS = 48;
+constexpr int GROUP_M = 8;                    // raster: 8 M-tiles per band
+constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 0.1 s for the abort drain
 
 // Instruction descriptor, kind::mxf4nvf4: A/B format E2M1 (1) at bits 7 and
 // 10, both K-major, N>>3 at bit 17, scale format UE4M3 (0) at bit 23, M>>4 at
-// bit 24, scale-factor ids 0, dense K = 64.
+// bit 24 (M = 256 across the pair), scale-factor ids 0, dense K = 64.
 constexpr uint32_t IDESC = (1u << 7) | (1u << 10) | (static_cast<uint32_t>(BN >> 3) << 17) |
                            (static_cast<uint32_t>(BM >> 4) << 24);
 
-enum : uint32_t { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u };
+enum : uint32_t { kFaultProducer = 1u, kFaultMma = 2u, kFaultEpilogue = 4u, kFaultScales = 8u };
 
 struct Params {
   int M, N, K;
@@ -76,8 +94,8 @@ struct Params {
   int y_fp32;
 };
 
-// Band rasterization: consecutive tiles walk GROUP_M M-blocks down one
-// N-column band, so the CTAs resident at one time share A and B tiles in L2.
+// Band rasterization: consecutive tiles walk GROUP_M M-tiles down one N band,
+// so the pairs resident at one time share A and B tiles in L2.
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int per_group = GROUP_M * p.num_n_blk;
   const int group = t / per_group;
@@ -88,18 +106,29 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int
   nb = r / gsize;
 }
 
+struct Abort {
+  volatile uint32_t* local;   // this CTA's flag
+  uint32_t peer_cluster;      // shared::cluster address of the peer's flag
+
+  __device__ __forceinline__ bool raised() const { return *local != 0u; }
+  __device__ __forceinline__ void raise(uint32_t who) const {
+    *local = 1u;
+    ptx::st_shared_cluster_u32(peer_cluster, 1u);
+    atomicOr(&g_fault_word, who);
+  }
+};
+
 // Bounded wait: true when the phase of parity `parity` completed; false when
-// another role aborted or the time limit passed (then this role aborts too).
-__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
-                                             volatile uint32_t* abort_flag, uint32_t who) {
+// the pair aborted or the time limit passed (then this role aborts the pair).
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, const Abort& ab,
+                                             uint32_t who) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
-    if (*abort_flag) return false;
+    if (ab.raised()) return false;
     if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1u;
-      atomicOr(&g_fault_word, who);
+      ab.raise(who);
       return false;
     }
   }
@@ -157,6 +186,41 @@ __device__ __forceinline__ void store_cols(const uint32_t (&r)[32], const Params
   }
 }
 
+// Tensor-memory columns of scale buffer `buf`: A's 16, then B's 32.
+__device__ __forceinline__ uint32_t sfa_cols(uint32_t tmem, uint32_t buf) {
+  return tmem + SF_COL + buf * SF_BUF_COLS;
+}
+__device__ __forceinline__ uint32_t sfb_cols(uint32_t tmem, uint32_t buf) {
+  return tmem + SF_COL + buf * SF_BUF_COLS + 16u;
+}
+
+// Copy half (`part` 0 or 1) of one stage's scale atoms into tensor-memory
+// buffer `buf` of both CTAs. Per K = 64 step j, A's 128 rows go to 4 columns
+// and B's 256 rows to 8 (row block h -> columns 4h..4h+3). Part 0: the 4 A
+// atoms and B row block 0 of steps 0-1; part 1: B row block 0 of steps 2-3
+// and row block 1 of all steps.
+__device__ __forceinline__ void copy_scales(uint32_t tmem, uint32_t ssfa, uint32_t ssfb,
+                                            uint32_t buf, int part) {
+  const uint32_t tsfa = sfa_cols(tmem, buf);
+  const uint32_t tsfb = sfb_cols(tmem, buf);
+  if (part == 0) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      ptx::tc_cp_32x128b_warpx4_pair(tsfa + 4u * j, ptx::smem_desc(ssfa + 512u * j, 0, 128, 0));
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+      ptx::tc_cp_32x128b_warpx4_pair(tsfb + 8u * j, ptx::smem_desc(ssfb + 512u * j, 0, 128, 0));
+  } else {
+#pragma unroll
+    for (int j = 2; j < 4; ++j)
+      ptx::tc_cp_32x128b_warpx4_pair(tsfb + 8u * j, ptx::smem_desc(ssfb + 512u * j, 0, 128, 0));
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      ptx::tc_cp_32x128b_warpx4_pair(tsfb + 8u * j + 4u,
+                                     ptx::smem_desc(ssfb + 2048u + 512u * j, 0, 128, 0));
+  }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSFA,
@@ -169,11 +233,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tmem_full = empty + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* sf_full = drain + 1;
+  uint64_t* sf_empty = sf_full + NSF;
+  uint64_t* drain_sf = sf_empty + NSF;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();   // 0 = even CTA (issues the MMAs)
+  const bool leader = (rank == 0);
+  const int pair = blockIdx.x >> 1;
+  const int num_pairs = gridDim.x >> 1;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -181,8 +252,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&empty[s], 1);
     }
     ptx::mbar_init(tmem_full, 1);
-    ptx::mbar_init(tmem_empty, NUM_EPI_WARPS);
+    ptx::mbar_init(tmem_empty, 2 * NUM_EPI_WARPS);
     ptx::mbar_init(drain, 1);
+    for (int b = 0; b < NSF; ++b) {
+      ptx::mbar_init(&sf_full[b], NUM_SF_WARPS);
+      ptx::mbar_init(&sf_empty[b], 1);
+    }
+    ptx::mbar_init(drain_sf, NUM_SF_WARPS);
     *abort_flag = 0u;
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tmA);
@@ -191,13 +267,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tma_prefetch_desc(&tmSFB);
   }
   if (warp == 1) {
-    ptx::tmem_alloc(tmem_holder, TMEM_COLS);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(tmem_holder, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  const Abort ab{abort_flag,
+                 ptx::mapa_shared(ptx::smem_u32(const_cast<uint32_t*>(abort_flag)), rank ^ 1u)};
   const int num_tiles = p.num_m_blk * p.num_n_blk;
 
   if (warp == 0) {
@@ -206,22 +284,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t pending = 0, pending_parity = 0;  // stages loaded, not yet seen free
       bool aborted = false;
-      for (int t = blockIdx.x; t < num_tiles && !aborted; t += gridDim.x) {
+      for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
         int mb, nb;
         tile_coords(t, p, mb, nb);
+        const int arow = mb * BM + static_cast<int>(rank) * HALF;
+        const int brow = nb * BN + static_cast<int>(rank) * HALF;
         for (int kt = 0; kt < p.num_k_tiles; ++kt) {
-          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer)) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, ab, kFaultProducer)) {
             aborted = true;
             break;
           }
           pending &= ~(1u << stage);
           uint8_t* st = smem + stage * STAGE_BYTES;
-          ptx::mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-          ptx::tma_load_2d(st, &tmA, &full[stage], kt * BK_BYTES, mb * BM);
-          ptx::tma_load_2d(st + A_BYTES, &tmB, &full[stage], kt * BK_BYTES, nb * BN);
-          ptx::tma_load_3d(st + A_BYTES + B_BYTES, &tmSFA, &full[stage], 0, kt * 4, mb);
-          ptx::tma_load_3d(st + A_BYTES + B_BYTES + SFA_BYTES, &tmSFB, &full[stage], 0, kt * 4,
-                           nb * 2);
+          // the even CTA's barrier counts both CTAs' bytes of this stage
+          const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(&full[stage]), 0);
+          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          ptx::tma_load_2d_pair(st, &tmA, bar, kt * BK_BYTES, arow);
+          ptx::tma_load_2d_pair(st + A_BYTES, &tmB, bar, kt * BK_BYTES, brow);
+          ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES, &tmSFA, bar, 0, kt * 4,
+                                mb * 2 + static_cast<int>(rank));
+          ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tmSFB, bar, 0, kt * 4, nb * 2);
           pending |= 1u << stage;
           pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == STAGES) {
@@ -230,77 +312,108 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       }
-      if (aborted) {
-        // let every issued copy land before the CTA can exit
+      if (aborted && leader) {
+        // let every issued copy of the pair land before the CTAs can exit
         for (int s = 0; s < STAGES; ++s)
           if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
       }
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer --
-    if (lane == 0) {
+    if (leader && lane == 0) {
       const uint32_t smem_base = ptx::smem_u32(smem);
-      uint32_t stage = 0, phase = 0, acc_phase = 0, sf_buf = 0;
+      uint32_t stage = 0, phase = 0, acc_phase = 0, sf_buf = 0, sf_phase = 0;
       bool aborted = false;
-      for (int t = blockIdx.x; t < num_tiles && !aborted; t += gridDim.x) {
-        if (!wait_bounded(tmem_empty, acc_phase ^ 1u, abort_flag, kFaultMma)) {
-          aborted = true;
-          break;
-        }
-        ptx::tc_fence_after();
+      for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
         for (int kt = 0; kt < p.num_k_tiles; ++kt) {
-          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma)) {
+          if (!wait_bounded(&full[stage], phase, ab, kFaultMma) ||
+              !wait_bounded(&sf_full[sf_buf], sf_phase, ab, kFaultMma)) {
             aborted = true;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t sa = smem_base + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          const uint32_t ssfa = sb + B_BYTES;
-          const uint32_t ssfb = ssfa + SFA_BYTES;
-          const uint32_t tsfa = tmem + SFA_COL + sf_buf * 16u;
-          const uint32_t tsfb = tmem + SFB_COL + sf_buf * 32u;
-          // scale atoms -> tensor memory: 4 columns per 128 rows per K=64 step
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ptx::tc_cp_32x128b_warpx4(tsfa + 4u * j, ptx::smem_desc(ssfa + 512u * j, 0, 128, 0));
-            ptx::tc_cp_32x128b_warpx4(tsfb + 8u * j, ptx::smem_desc(ssfb + 512u * j, 0, 128, 0));
-            ptx::tc_cp_32x128b_warpx4(tsfb + 8u * j + 4u,
-                                      ptx::smem_desc(ssfb + 2048u + 512u * j, 0, 128, 0));
+          if (kt == 0) {
+            // the accumulator must have been drained by both epilogues
+            if (!wait_bounded(tmem_empty, acc_phase ^ 1u, ab, kFaultMma)) {
+              aborted = true;
+              break;
+            }
+            ptx::tc_fence_after();
           }
+          const uint32_t tsfa = sfa_cols(tmem, sf_buf);
+          const uint32_t tsfb = sfb_cols(tmem, sf_buf);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint64_t adesc = ptx::smem_desc(sa + 32u * j, 16, 1024, 2);
             const uint64_t bdesc = ptx::smem_desc(sb + 32u * j, 16, 1024, 2);
-            ptx::tc_mma_nvf4(tmem + ACC_COL, adesc, bdesc, IDESC, tsfa + 4u * j, tsfb + 8u * j,
-                             (kt | j) != 0 ? 1u : 0u);
+            ptx::tc_mma_nvf4_pair(tmem + ACC_COL, adesc, bdesc, IDESC, tsfa + 4u * j,
+                                  tsfb + 8u * j, (kt | j) != 0 ? 1u : 0u);
           }
-          ptx::tc_commit(&empty[stage]);  // frees the stage when these MMAs finish
-          sf_buf ^= 1u;
+          ptx::tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
+          ptx::tc_commit_pair_mc(&sf_empty[sf_buf], 0x1);  // frees the scale buffer
+          if (++sf_buf == NSF) {
+            sf_buf = 0;
+            sf_phase ^= 1u;
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (aborted) break;
-        ptx::tc_commit(tmem_full);  // accumulator ready when all MMAs finish
+        ptx::tc_commit_pair_mc(tmem_full, 0x3);  // accumulators ready in both CTAs
         acc_phase ^= 1u;
       }
       if (aborted) {
-        ptx::tc_commit(drain);
+        ptx::tc_commit_pair_mc(drain, 0x1);
         drain_wait(drain, 0);
+      }
+    }
+  } else if (warp < EPI_WARP0) {
+    // ----------------------------------------------------- scale-copy warps --
+    if (leader && lane == 0) {
+      const uint32_t smem_base = ptx::smem_u32(smem);
+      uint32_t stage = 0, phase = 0, sf_buf = 0, sf_phase = 0;
+      bool aborted = false;
+      for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
+        for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+          if (!wait_bounded(&full[stage], phase, ab, kFaultScales) ||
+              !wait_bounded(&sf_empty[sf_buf], sf_phase ^ 1u, ab, kFaultScales)) {
+            aborted = true;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t ssfa = smem_base + stage * STAGE_BYTES + A_BYTES + B_BYTES;
+          copy_scales(tmem, ssfa, ssfa + SFA_BYTES, sf_buf, warp - SF_WARP0);
+          ptx::tc_commit_pair_mc(&sf_full[sf_buf], 0x1);  // buffer ready when copies land
+          if (++sf_buf == NSF) {
+            sf_buf = 0;
+            sf_phase ^= 1u;
+          }
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (aborted) {
+        ptx::tc_commit_pair_mc(drain_sf, 0x1);
+        drain_wait(drain_sf, 0);
       }
     }
   } else {
     // -------------------------------------------------------------- epilogue --
-    const int q = warp & 3;                 // tensor-memory lane quarter
-    const int half = (warp - 2) >> 2;       // accumulator columns [128*half, +128)
+    const int q = warp & 3;                     // tensor-memory lane quarter
+    const int half = (warp - EPI_WARP0) >> 2;   // accumulator columns [128*half, +128)
     const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
+    const uint32_t release = ptx::mapa_shared(ptx::smem_u32(tmem_empty), 0);
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+    for (int t = pair; t < num_tiles; t += num_pairs) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
-      if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue)) break;
+      if (!wait_bounded(tmem_full, acc_phase, ab, kFaultEpilogue)) break;
       ptx::tc_fence_after();
       uint32_t r0[32], r1[32], r2[32], r3[32];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128u;
@@ -311,10 +424,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::tc_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(tmem_empty);
+      if (lane == 0) ptx::mbar_arrive_cluster(release);
       acc_phase ^= 1u;
 
-      const int64_t row = static_cast<int64_t>(mb) * BM + q * 32 + lane;
+      const int64_t row = static_cast<int64_t>(mb) * BM + rank * HALF + q * 32 + lane;
       if (row >= p.M) continue;
       const int col0 = nb * BN + half * 128;
       store_cols(r0, p, row, col0 + 0, alpha);
@@ -325,11 +438,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 
   ptx::tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  ptx::cluster_sync();  // neither CTA frees tensor memory while the pair works
   ptx::tc_fence_after();
   if (warp == 1) {
     __syncwarp();
-    ptx::tmem_dealloc(tmem, TMEM_COLS);
+    ptx::tmem_dealloc_pair(tmem, TMEM_COLS);
   }
 }
 

@@ -294,10 +294,10 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
 
   CUtensorMap tmA, tmB, tmSFA, tmSFB;
   if (nvfp4_status e = encode_2d(enc, &tmA, a_codes, static_cast<uint64_t>(k / 2),
-                                 static_cast<uint64_t>(m), BM))
+                                 static_cast<uint64_t>(m), HALF))
     return e;
   if (nvfp4_status e = encode_2d(enc, &tmB, b_codes, static_cast<uint64_t>(k / 2),
-                                 static_cast<uint64_t>(n), BN))
+                                 static_cast<uint64_t>(n), HALF))
     return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFA, a_sf, m, k, 1u)) return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFB, b_sf, n, k, 2u)) return e;
@@ -327,9 +327,26 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   p.y_fp32 = y_dtype;
   const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
   if (tiles >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;
-  const int grid = static_cast<int>(tiles < st->sms ? tiles : st->sms);
-  gemm_kernel<<<grid, NUM_THREADS, SMEM_BYTES, reinterpret_cast<cudaStream_t>(stream)>>>(
-      tmA, tmB, tmSFA, tmSFB, p);
+  // one CTA pair (cluster of 2 SMs) per 256x256 tile at a time, persistent
+  const int64_t max_pairs = st->sms / 2;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmSFA, tmSFB, p) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
   return launch_status();
 }
 
