@@ -31,7 +31,12 @@
 //   warps 4..11  epilogue (both CTAs): two warps per tensor-memory lane
 //           quarter drain 128 columns each into registers, release the
 //           accumulator (arrive on the even CTA's barrier), then scale by
-//           1/(g_a g_b), convert and store.
+//           1/(g_a g_b), convert, and write 32-row x 64-byte chunks into a
+//           double-buffered swizzled shared-memory tile that a TMA bulk
+//           tensor store copies out (full-line writes, ragged edges clipped
+//           by the TMA unit). Per-thread 16-byte stores of whole rows would
+//           cost one L2 sector write each and steal L2 bandwidth from the
+//           operand loads.
 // Every mbarrier wait is bounded in time; on expiry the kernel records a fault
 // word, both CTAs of the pair stop, in-flight copies and MMAs are drained
 // (again with a bound) and tensor memory is released before the CTAs exit.
@@ -72,7 +77,11 @@ constexpr int NSF = 4;                        // tensor-memory scale buffers
 constexpr uint32_t SF_COL = 256;              // NSF x 48 columns: [A 16 | B 32]
 constexpr uint32_t SF_BUF_COLS = 48;
 constexpr int GROUP_M = 8;                    // raster: 8 M-tiles per band
-constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
+constexpr int EPI_CHUNK_BYTES = 32 * 64;      // 32 rows x 64 bytes, 64-byte swizzle
+constexpr int EPI_WARP_BYTES = 2 * EPI_CHUNK_BYTES;
+constexpr int EPI_OFF = STAGES * STAGE_BYTES;  // staging tiles after the ring
+constexpr int BAR_OFF = EPI_OFF + NUM_EPI_WARPS * EPI_WARP_BYTES;
+constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(BAR_OFF) + 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 0.1 s for the abort drain
 
@@ -142,48 +151,38 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Scale 32 accumulator columns of one output row by alpha and store them
-// (bf16 or fp32), 16-byte vectors where the whole vector is inside N.
-__device__ __forceinline__ void store_cols(const uint32_t (&r)[32], const Params& p, int64_t row,
-                                           int col0, float alpha) {
-  if (p.y_fp32) {
-    float* yrow = reinterpret_cast<float*>(p.y) + row * p.ldy;
+// Write 64 bytes of this thread's output row into a 32-row x 64-byte staging
+// chunk with the 64-byte swizzle (16-byte unit u of row r at u ^ ((r>>1)&3)),
+// which the TMA store undoes and which spreads a warp's 32 rows over all
+// banks. bf16: 32 accumulator columns; fp32: the 16 starting at `off`.
+__device__ __forceinline__ void stage_bf16(uint32_t chunk, int row, const uint32_t (&r)[32],
+                                           float alpha) {
+  const uint32_t base = chunk + row * 64;
+  const int sw = (row >> 1) & 3;
 #pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      const int col = col0 + v * 4;
-      float o[4];
+  for (int u = 0; u < 4; ++u) {
+    uint32_t w[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) o[e] = __uint_as_float(r[v * 4 + e]) * alpha;
-      if (col + 4 <= p.N) {
-        *reinterpret_cast<float4*>(yrow + col) = make_float4(o[0], o[1], o[2], o[3]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (col + e < p.N) yrow[col + e] = o[e];
-      }
+    for (int e = 0; e < 4; ++e) {
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[u * 8 + 2 * e]) * alpha,
+                                                      __uint_as_float(r[u * 8 + 2 * e + 1]) * alpha);
+      w[e] = *reinterpret_cast<const uint32_t*>(&b2);
     }
-  } else {
-    uint16_t* yrow = reinterpret_cast<uint16_t*>(p.y) + row * p.ldy;
-#pragma unroll
-    for (int v = 0; v < 4; ++v) {
-      const int col = col0 + v * 8;
-      uint32_t packed[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[v * 8 + 2 * e]) * alpha,
-                                                        __uint_as_float(r[v * 8 + 2 * e + 1]) * alpha);
-        packed[e] = *reinterpret_cast<const uint32_t*>(&b2);
-      }
-      if (col + 8 <= p.N) {
-        *reinterpret_cast<uint4*>(yrow + col) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          if (col + e < p.N)
-            yrow[col + e] = static_cast<uint16_t>((packed[e >> 1] >> (16 * (e & 1))) & 0xFFFFu);
-      }
-    }
+    ptx::st_shared_v4(base + ((u ^ sw) << 4), w[0], w[1], w[2], w[3]);
   }
+}
+
+__device__ __forceinline__ void stage_f32(uint32_t chunk, int row, const uint32_t (&r)[32],
+                                          int off, float alpha) {
+  const uint32_t base = chunk + row * 64;
+  const int sw = (row >> 1) & 3;
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+    ptx::st_shared_v4(base + ((u ^ sw) << 4),
+                      __float_as_uint(__uint_as_float(r[off + 4 * u + 0]) * alpha),
+                      __float_as_uint(__uint_as_float(r[off + 4 * u + 1]) * alpha),
+                      __float_as_uint(__uint_as_float(r[off + 4 * u + 2]) * alpha),
+                      __float_as_uint(__uint_as_float(r[off + 4 * u + 3]) * alpha));
 }
 
 // Tensor-memory columns of scale buffer `buf`: A's 16, then B's 32.
@@ -224,11 +223,12 @@ __device__ __forceinline__ void copy_scales(uint32_t tmem, uint32_t ssfa, uint32
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const __grid_constant__ CUtensorMap tmSFA,
-                const __grid_constant__ CUtensorMap tmSFB, const Params p) {
+                const __grid_constant__ CUtensorMap tmSFB,
+                const __grid_constant__ CUtensorMap tmY, const Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + BAR_OFF);
   uint64_t* empty = full + STAGES;
   uint64_t* tmem_full = empty + STAGES;
   uint64_t* tmem_empty = tmem_full + 1;
@@ -265,6 +265,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tma_prefetch_desc(&tmB);
     ptx::tma_prefetch_desc(&tmSFA);
     ptx::tma_prefetch_desc(&tmSFB);
+    ptx::tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -409,6 +410,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - EPI_WARP0) >> 2;   // accumulator columns [128*half, +128)
     const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
     const uint32_t release = ptx::mapa_shared(ptx::smem_u32(tmem_empty), 0);
+    uint8_t* const stage_tiles = smem + EPI_OFF + (warp - EPI_WARP0) * EPI_WARP_BYTES;
+    uint32_t nchunk = 0;  // chunks this warp has handed to the TMA (buffer = nchunk & 1)
+    // Hand one staged chunk to the TMA once the buffer's previous store has
+    // finished reading it.
+    auto emit = [&](auto&& fill, int x, int y) {
+      uint8_t* buf = stage_tiles + (nchunk & 1u) * EPI_CHUNK_BYTES;
+      if (lane == 0) ptx::bulk_wait_group_read<1>();
+      __syncwarp();
+      fill(ptx::smem_u32(buf));
+      ptx::fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        ptx::tma_store_2d(&tmY, buf, x, y);
+        ptx::bulk_commit_group();
+      }
+      ++nchunk;
+    };
     uint32_t acc_phase = 0;
     for (int t = pair; t < num_tiles; t += num_pairs) {
       int mb, nb;
@@ -427,14 +445,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (lane == 0) ptx::mbar_arrive_cluster(release);
       acc_phase ^= 1u;
 
-      const int64_t row = static_cast<int64_t>(mb) * BM + rank * HALF + q * 32 + lane;
-      if (row >= p.M) continue;
+      const int row0 = mb * BM + static_cast<int>(rank) * HALF + q * 32;  // this warp's rows
+      if (row0 >= p.M) continue;  // warp-uniform; rows past M inside are clipped by the TMA
       const int col0 = nb * BN + half * 128;
-      store_cols(r0, p, row, col0 + 0, alpha);
-      store_cols(r1, p, row, col0 + 32, alpha);
-      store_cols(r2, p, row, col0 + 64, alpha);
-      store_cols(r3, p, row, col0 + 96, alpha);
+      if (!p.y_fp32) {
+        emit([&](uint32_t b) { stage_bf16(b, lane, r0, alpha); }, col0 + 0, row0);
+        emit([&](uint32_t b) { stage_bf16(b, lane, r1, alpha); }, col0 + 32, row0);
+        emit([&](uint32_t b) { stage_bf16(b, lane, r2, alpha); }, col0 + 64, row0);
+        emit([&](uint32_t b) { stage_bf16(b, lane, r3, alpha); }, col0 + 96, row0);
+      } else {
+        emit([&](uint32_t b) { stage_f32(b, lane, r0, 0, alpha); }, col0 + 0, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r0, 16, alpha); }, col0 + 16, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r1, 0, alpha); }, col0 + 32, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r1, 16, alpha); }, col0 + 48, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r2, 0, alpha); }, col0 + 64, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r2, 16, alpha); }, col0 + 80, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r3, 0, alpha); }, col0 + 96, row0);
+        emit([&](uint32_t b) { stage_f32(b, lane, r3, 16, alpha); }, col0 + 112, row0);
+      }
     }
+    if (lane == 0) ptx::bulk_wait_group_all();  // stores done before the CTA can exit
   }
 
   ptx::tc_fence_before();

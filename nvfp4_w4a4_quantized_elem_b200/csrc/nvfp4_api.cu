@@ -251,6 +251,22 @@ nvfp4_status encode_2d(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+// Output for TMA stores: [m][ldy] of bf16 / fp32, boxes of 32 rows x 64 bytes
+// with the 64-byte swizzle the epilogue's staging tiles use.
+nvfp4_status encode_y(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, void* base,
+                      int64_t m, int64_t n, int64_t ldy, int y_dtype) {
+  const uint64_t esize = y_dtype == 0 ? 2u : 4u;
+  cuuint64_t dims[2] = {static_cast<uint64_t>(n), static_cast<uint64_t>(m)};
+  cuuint64_t strides[1] = {static_cast<uint64_t>(ldy) * esize};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(64u / esize), 32u};
+  cuuint32_t estr[2] = {1u, 1u};
+  CUresult r = enc(map, y_dtype == 0 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32,
+                   2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
+
 // Scale factors as [row blocks][atoms][128 x uint32]: one box = whole atoms.
 nvfp4_status encode_sf(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, const void* base,
                        int64_t rows, int64_t k, uint32_t box_row_blocks) {
@@ -292,7 +308,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (nvfp4_status e = get_encoder(&enc)) return e;
 
-  CUtensorMap tmA, tmB, tmSFA, tmSFB;
+  CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
   if (nvfp4_status e = encode_2d(enc, &tmA, a_codes, static_cast<uint64_t>(k / 2),
                                  static_cast<uint64_t>(m), HALF))
     return e;
@@ -301,6 +317,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
     return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFA, a_sf, m, k, 1u)) return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFB, b_sf, n, k, 2u)) return e;
+  if (nvfp4_status e = encode_y(enc, &tmY, y, m, n, ldy, y_dtype)) return e;
 
   {
     std::lock_guard<std::mutex> lock(g_mutex);
@@ -343,7 +360,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmSFA, tmSFB, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmSFA, tmSFB, tmY, p) != cudaSuccess) {
     cudaGetLastError();
     return NVFP4_ERR_CUDA;
   }
