@@ -10,13 +10,19 @@
 //   amax_kernel      one pass over x, one partial max per CTA (no atomics, so
 //                    the workspace needs no initialisation);
 //   quantize_kernel  every CTA first reduces the partials to g (a few hundred
-//                    floats from L2), then quantizes. A warp task is one
-//                    (128-row block, row l in 0..31, 4 consecutive 64-column
-//                    atoms): the warp reads rows l, l+32, l+64, l+96 — four
-//                    full 128-byte lines per atom — so each lane holds 8
-//                    elements (half a 16-element block) and the 4 row groups
-//                    x 4 blocks of scales form one whole 16-byte line of the
-//                    swizzled scale atom, written with a single store.
+//                    floats from L2) and tabulates r(s) = g / dec(s) for all
+//                    128 E4M3 codes (one IEEE division each, so the per-block
+//                    division becomes a shared-memory load with the same
+//                    result), then quantizes. A warp task is one (128-row
+//                    block, row l in 0..31, 4 consecutive 64-column atoms):
+//                    the warp reads rows l, l+32, l+64, l+96 — four full
+//                    128-byte lines per atom — so each lane holds 8 elements
+//                    (half a 16-element block) and the 4 row groups x 4 blocks
+//                    of scales form one 16-byte line of the swizzled atom.
+// amax_b / 6 is computed as q = amax_b * RN(1/6), q + RN((amax_b - 6 q) *
+// RN(1/6)) with two FMAs; this equals the IEEE quotient for every
+// non-negative bf16 value (checked exhaustively with exact rationals in the
+// test-suite), which is the only input it ever sees.
 #pragma once
 
 #include "ptx.cuh"
@@ -30,6 +36,14 @@ constexpr int kMaxPartials = 4096;            // workspace = 16 KiB
 constexpr int kQuantThreads = 256;
 constexpr int kQuantBlocksPerSM = 8;
 constexpr int kAtomsPerTask = 4;
+constexpr float kInv6 = 0.16666667163372039794921875f;  // RN(1/6) = 0x3E2AAAAB
+
+// RN(a / 6) for a non-negative bf16 value a (see the header comment).
+__device__ __forceinline__ float div6_rn(float a) {
+  const float q = __fmul_rn(a, kInv6);
+  const float r = __fmaf_rn(-q, 6.0f, a);
+  return __fmaf_rn(r, kInv6, q);
+}
 
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 v;
@@ -55,7 +69,21 @@ __global__ void __launch_bounds__(kAmaxThreads)
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int64_t chunks = k >> 3;  // 16-byte chunks per row
   uint32_t m = 0;
-  for (int64_t r = warp; r < rows; r += nwarps) {
+  if (ldx == k) {
+    // contiguous tensor: one flat stream of 16-byte chunks, 8 loads in flight
+    const int64_t total = rows * chunks;
+    const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    for (; i + 7 * nthreads < total; i += 8 * nthreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = ldg_stream(x + (i + u * nthreads) * 8);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) m = max(m, absmax_bits8(v[u]));
+    }
+    for (; i < total; i += nthreads) m = max(m, absmax_bits8(ldg_stream(x + i * 8)));
+  }
+  for (int64_t r = (ldx == k) ? rows : warp; r < rows; r += nwarps) {
     const uint16_t* row = x + r * ldx;
     int64_t c = lane;
     for (; c + 96 < chunks; c += 128) {
@@ -95,6 +123,7 @@ __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w 
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs a) {
   __shared__ float s_g;
+  __shared__ float s_rtab[128];
   __shared__ uint32_t s_red[kQuantThreads / 32];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -121,6 +150,11 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
   __syncthreads();
   const float g = s_g;
   if (blockIdx.x == 0 && threadIdx.x == 0) *a.global_out = g;
+  if (threadIdx.x < 128) {
+    const float ds = ptx::e4m3_value(threadIdx.x);
+    s_rtab[threadIdx.x] = (ds == 0.0f) ? 0.0f : __fdiv_rn(g, ds);  // r = 0 keeps only signs
+  }
+  __syncthreads();
 
   // ---- blocks ----------------------------------------------------------------
   const int64_t n_rb = (a.rows + 127) / 128;
@@ -160,10 +194,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
       uint32_t mb = absmax_bits8(v[u]);
       mb = max(mb, __shfl_xor_sync(0xFFFFFFFFu, mb, 1));
       const float amax_b = __uint_as_float(mb << 16);
-      const float t6 = __fdiv_rn(amax_b, 6.0f);
-      const uint32_t s = ptx::cvt_e4m3(__fmul_rn(t6, g));
-      const float ds = ptx::e4m3_value(s);
-      const float r = (ds == 0.0f) ? 0.0f : __fdiv_rn(g, ds);  // r = 0 keeps only signs
+      const uint32_t s = ptx::cvt_e4m3(__fmul_rn(div6_rn(amax_b), g));
+      const float r = s_rtab[s];
 
       float f[8];
       f[0] = __fmul_rn(bf16_lo(v[u].x), r);
@@ -177,20 +209,14 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
       const uint32_t packed = ptx::cvt_e2m1x8(f);
       if (ok) *reinterpret_cast<uint32_t*>(a.codes + row * half_k + (col >> 1)) = packed;
 
-      // scales: lanes 8g+{0,2,4,6} hold blocks 0..3 of row group g
-      const int base = grp * 8;
-      const uint32_t b0 = __shfl_sync(0xFFFFFFFFu, s, base + 0);
-      const uint32_t b1 = __shfl_sync(0xFFFFFFFFu, s, base + 2);
-      const uint32_t b2 = __shfl_sync(0xFFFFFFFFu, s, base + 4);
-      const uint32_t b3 = __shfl_sync(0xFFFFFFFFu, s, base + 6);
-      const uint32_t word = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
-      const uint32_t w0 = __shfl_sync(0xFFFFFFFFu, word, 0);
-      const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, word, 8);
-      const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, word, 16);
-      const uint32_t w3 = __shfl_sync(0xFFFFFFFFu, word, 24);
-      if (lane == 0)
-        *reinterpret_cast<uint4*>(a.sf + (rb * n_ka + ka) * 512 + l * 16) =
-            make_uint4(w0, w1, w2, w3);
+      // scales: lanes 8g+{2b, 2b+1} hold block b of row group g; OR the 4
+      // blocks' bytes into one word per group, whose 4 words are the 16
+      // contiguous bytes of line l of the atom
+      uint32_t word = s << (8 * (j >> 1));
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 2);
+      word |= __shfl_xor_sync(0xFFFFFFFFu, word, 4);
+      if (j == 0)
+        *reinterpret_cast<uint32_t*>(a.sf + (rb * n_ka + ka) * 512 + l * 16 + grp * 4) = word;
     }
   }
 }

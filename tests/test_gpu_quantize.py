@@ -62,6 +62,20 @@ def test_quantize_every_bf16_value(nv, orc):
         check(nv, orc, x, gin, what=f"all-bf16 g={gin}")
 
 
+def test_quantize_every_bf16_as_block_amax(nv, orc):
+    """One block per non-negative finite bf16 value v = [v, -v/2, 0, ...]:
+    every possible block amax goes through the scale computation, under
+    globals that put amax/6*g across the whole E4M3 range."""
+    b = np.arange(0, 0x7F80, dtype=np.uint32)
+    v = (b << 16).view(np.float32)
+    x = np.zeros((len(v), 16), np.float32)
+    x[:, 0] = v
+    x[:, 1] = -v / 2
+    xb = torch.from_numpy(x).to(torch.bfloat16)
+    for gin in (1.0, 2.0 ** 100, 2.0 ** -100, 3.0, 1e30):
+        check(nv, orc, xb, gin, what=f"block amax sweep g={gin}")
+
+
 def test_quantize_each_block_scale_path(nv, orc):
     # blocks whose amax spans the whole E4M3 range relative to one global,
     # including subnormal and zero scales (signed-zero codes)
