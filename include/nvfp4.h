@@ -121,8 +121,8 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
  * Arguments, layouts, results and errors are those of nvfp4_quantize (minus
  * the workspace pair). Additionally:
  *   - NVFP4_ERR_UNSUPPORTED if the amax pass would need more than
- *     NVFP4_NOALLOC_MAX_PARTIALS CTAs (it launches min(ceil(rows/32),
- *     2 x SM count) of them; 296 on a 148-SM B200).
+ *     NVFP4_NOALLOC_MAX_PARTIALS CTAs (it launches at most 2 x SM count of
+ *     them; 296 on a 148-SM B200).
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture. Later calls allocate nothing and call no
@@ -140,8 +140,29 @@ nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k,
                                     uint8_t* codes, uint8_t* sf,
                                     float* global_out, nvfp4_stream_t stream);
 
-/* Workspace bytes nvfp4_gemm needs (0 for every shape the current kernels
- * handle; kept so callers need not change when split-K arrives). */
+/*
+ * nvfp4_calibrate_global — one step of static (calibrated) global-scale
+ * calibration: the pages calibrate activation scales offline on a frozen set
+ * of 128 samples x 32K tokens (news §03, reading §4.1) and then serve with
+ * those fixed scales. Folds one calibration batch into a running maximum and
+ * writes the global scale that the running maximum implies:
+ *   *running_amax = max(*running_amax, max |x|);
+ *   *global_out   = 2688 / *running_amax (1 if that is 0 or not finite).
+ * Start with *running_amax = 0; pass *global_out as nvfp4_quantize's
+ * global_in (static mode) afterwards.
+ *   x, rows, k, ldx, workspace, workspace_bytes: as nvfp4_quantize (dynamic).
+ *   running_amax, global_out: device FP32 scalars (4-byte aligned).
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED (k % 16), CUDA.
+ */
+nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k,
+                                    int64_t ldx, float* running_amax,
+                                    float* global_out, void* workspace,
+                                    size_t workspace_bytes,
+                                    nvfp4_stream_t stream);
+
+/* Workspace bytes nvfp4_gemm can use: m*n*4 for m <= 64 (few-token GEMMs
+ * split K across CTAs and sum FP32 partials there), else 0. Passing less (or
+ * NULL) is allowed and only disables the split. */
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -159,6 +180,10 @@ size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *   m, n     >= 1.   k: k % 32 == 0 (TMA row pitch k/2 must be a multiple of
  *            16 bytes) and k >= 32.
  *   a_codes, b_codes: 16-byte aligned. a_sf, b_sf: 16-byte aligned.
+ *   workspace  device scratch, nvfp4_gemm_workspace_bytes(m,n,k) bytes,
+ *              16-byte aligned, or NULL; contents need no initialisation.
+ * m <= 64 runs the few-token kernel (weights on the MMA's 128-row side,
+ * tokens as its N); larger m the paired-CTA 256x256-tile kernel.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
  */
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
@@ -167,6 +192,36 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
                         int y_dtype, int64_t ldy, int64_t m, int64_t n,
                         int64_t k, void* workspace, size_t workspace_bytes,
                         nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm_swiglu_quant — gate_up projection of a W4A4 gated MLP with the
+ * activation and the next layer's activation quantization fused into the
+ * GEMM epilogue. Every linear layer of the recipe is W4A4 (news §03), so the
+ * MLP's hidden state h = silu(gate) * up is quantized right away for the down
+ * projection; here it never goes to memory in bf16. Computes, bit for bit,
+ *   Y  = nvfp4_gemm(A, B) in bf16 (gate and up halves),
+ *   h  = nvfp4_silu_mul(Y),
+ *   (h_codes, h_sf) = nvfp4_quantize(h, global_in = h_global)   [static]
+ * without writing Y or h.
+ *   A       activations [m][k] NVFP4 (codes, sf, global) as for nvfp4_gemm.
+ *   B       gate_up weights [2*ffn][k] NVFP4 with rows interleaved in blocks
+ *           of 128: rows [256b, 256b+128) = gate rows [128b, 128b+128),
+ *           rows [256b+128, 256b+256) = up rows [128b, 128b+128).
+ *   h_global  device FP32 static global of h (e.g. from
+ *           nvfp4_calibrate_global over calibration batches of h).
+ *   h_codes device [m][ffn/2] bytes, 16-byte aligned.
+ *   h_sf    device nvfp4_sf_bytes(m, ffn) bytes, 16-byte aligned; every byte
+ *           is written.
+ *   ffn % 128 == 0, k % 32 == 0.
+ * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
+ */
+nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf,
+                                     const float* a_global,
+                                     const uint8_t* b_codes, const uint8_t* b_sf,
+                                     const float* b_global, const float* h_global,
+                                     uint8_t* h_codes, uint8_t* h_sf, int64_t m,
+                                     int64_t ffn, int64_t k,
+                                     nvfp4_stream_t stream);
 
 /*
  * nvfp4_fuse_group_scales — global-scale repair of a fused module group

@@ -1,0 +1,383 @@
+// gemm_skinny.cuh — the W4A4 GEMM for few tokens (M <= 64): decode steps.
+//
+// Same product as gemm_sm100.cuh (Y = dequant(A) dequant(B)^T / (g_a g_b)),
+// computed as Y^T = B A^T so that the weights fill the 128-row MMA side and
+// the tokens are the MMA N (16..256): the tensor cores then do no work on
+// padded token rows, and the kernel streams the weights at memory speed.
+// News article "Qwen3.8-27B最激进4bit量化开源，权重显存暴降2.9倍！" §02
+// (W4A4 on 4-bit tensor cores); decode throughput is one of the serving
+// numbers the pages report (§04).
+//
+// One CTA per SM, persistent over work units (128 weight rows x one slice of
+// K). When the weight tiles alone cannot occupy the GPU, K is split across
+// CTAs and each slice adds its FP32 partial into a zeroed workspace with
+// red.global.add; a finalize kernel converts the sum.
+//   warp 0     TMA producer: W tile (128 rows x 128 B, 128-byte swizzle), the
+//              token tile (BNT rows), and both tiles' scale atoms, into a
+//              ring of up to 8 stages.
+//   warp 1     allocates tensor memory; one thread issues 4 MMAs
+//              (kind::mxf4nvf4.block16, M = 128, N = BNT, K = 64) per k-tile.
+//   warps 2-3  copy the stage's scale atoms into one of 4 tensor-memory scale
+//              buffers (tcgen05.cp 32x128b.warpx4, ~50 cycles each whatever
+//              the size): with only ~18 KiB of weights per k-tile the copies
+//              would otherwise set the pace of the weight stream.
+//   warps 4-7  epilogue: each thread owns one weight row (= one output
+//              column n) and drains its BNT token values 32 at a time; for a
+//              fixed token the 32 lanes write 32 consecutive columns.
+// Every wait is bounded; on expiry the fault word is set, copies and MMAs in
+// flight are drained (bounded) and tensor memory is freed before exit.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "fault.cuh"
+#include "ptx.cuh"
+
+namespace nvfp4 {
+
+namespace skinny {
+
+constexpr int BW = 128;           // weight rows per tile (MMA M)
+constexpr int BK = 256;           // FP4 elements per k-tile
+constexpr int BK_BYTES = BK / 2;
+constexpr int NUM_THREADS = 256;
+constexpr int SF_WARP0 = 2;       // warps 2, 3 copy scales
+constexpr int EPI_WARP0 = 4;      // warps 4..7 drain the accumulator
+constexpr int NSF = 4;            // tensor-memory scale buffers
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL = 256;  // NSF x 48 columns after the accumulator
+constexpr uint32_t SF_BUF_COLS = 48;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 100000000ull;
+constexpr size_t kSmemBudget = 220 * 1024;
+
+enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, kFaultScales = 128u };
+
+template <int BNT>
+struct Cfg {
+  static_assert(BNT == 16 || BNT == 32 || BNT == 64 || BNT == 128 || BNT == 256, "token tile");
+  static constexpr int A_BYTES = BW * BK_BYTES;             // 16 KiB of weights
+  static constexpr int B_BYTES = (BNT < 8 ? 8 : BNT) * BK_BYTES;
+  static constexpr int SFB_BLOCKS = (BNT + 127) / 128;      // 128-row scale blocks of tokens
+  static constexpr int SFA_BYTES = 2048;
+  static constexpr int SFB_BYTES = 2048 * SFB_BLOCKS;
+  static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
+  static constexpr int STAGES_FIT = static_cast<int>(kSmemBudget / STAGE_BYTES);
+  static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
+  static constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
+  static constexpr uint32_t SFB_COLS = 4u * SFB_BLOCKS;     // per K = 64 step
+  // kind::mxf4nvf4, E2M1 x E2M1, both K-major, N = BNT, UE4M3 scales, M = 128
+  static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) |
+                                    (static_cast<uint32_t>(BNT >> 3) << 17) |
+                                    (static_cast<uint32_t>(BW >> 4) << 24);
+};
+
+struct Params {
+  int M, N, K;              // Y is [M][N]; weights are [N][K], tokens [M][K]
+  int num_w_tiles, num_k_tiles, splits, k_tiles_per_split;
+  const float* a_global;    // tokens' global
+  const float* b_global;    // weights' global
+  void* y;                  // direct mode: [M][ldy] bf16 / fp32
+  int64_t ldy;
+  int y_fp32;
+  float* partial;           // split mode: [M][N] FP32, zeroed before launch
+};
+
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
+                                             volatile uint32_t* abort_flag, uint32_t who) {
+  if (ptx::mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1u;
+      atomicOr(&g_fault_word, who);
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait(bar, parity)) {
+    if (ptx::globaltimer_ns() - t0 > kDrainLimitNs) return;
+  }
+}
+
+__device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+
+__device__ __forceinline__ void red_add_f32(float* p, float v) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
+}
+
+template <int BNT>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
+                  const __grid_constant__ CUtensorMap tmSFW,
+                  const __grid_constant__ CUtensorMap tmSFX, const Params p) {
+  using C = Cfg<BNT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
+  uint64_t* empty = full + C::STAGES;
+  uint64_t* tmem_full = empty + C::STAGES;
+  uint64_t* tmem_empty = tmem_full + 1;
+  uint64_t* drain = tmem_empty + 1;
+  uint64_t* sf_full = drain + 1;
+  uint64_t* sf_empty = sf_full + NSF;
+  uint64_t* drain_sf = sf_empty + NSF;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
+  volatile uint32_t* abort_flag = tmem_holder + 1;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(tmem_full, 1);
+    ptx::mbar_init(tmem_empty, 4);
+    ptx::mbar_init(drain, 1);
+    for (int b = 0; b < NSF; ++b) {
+      ptx::mbar_init(&sf_full[b], 2);
+      ptx::mbar_init(&sf_empty[b], 1);
+    }
+    ptx::mbar_init(drain_sf, 2);
+    *abort_flag = 0u;
+    ptx::fence_mbarrier_init();
+    ptx::tma_prefetch_desc(&tmW);
+    ptx::tma_prefetch_desc(&tmX);
+    ptx::tma_prefetch_desc(&tmSFW);
+    ptx::tma_prefetch_desc(&tmSFX);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_holder, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const int num_units = p.num_w_tiles * p.splits;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer --
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0;
+      bool aborted = false;
+      for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+        const int wt = u % p.num_w_tiles, sp = u / p.num_w_tiles;
+        const int k0 = sp * p.k_tiles_per_split;
+        const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
+        for (int kt = k0; kt < k1; ++kt) {
+          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer)) {
+            aborted = true;
+            break;
+          }
+          pending &= ~(1u << stage);
+          uint8_t* st = smem + stage * C::STAGE_BYTES;
+          ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
+          ptx::tma_load_2d(st, &tmW, &full[stage], kt * BK_BYTES, wt * BW);
+          ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], kt * BK_BYTES, 0);
+          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, kt * 4, wt);
+          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
+                           kt * 4, 0);
+          pending |= 1u << stage;
+          pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (aborted)
+        for (int s = 0; s < C::STAGES; ++s)
+          if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------------------------- MMA issuer --
+    if (lane == 0) {
+      const uint32_t smem_base = ptx::smem_u32(smem);
+      uint32_t stage = 0, phase = 0, acc_phase = 0, sf_buf = 0, sf_phase = 0;
+      bool aborted = false;
+      for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+        const int sp = u / p.num_w_tiles;
+        const int k0 = sp * p.k_tiles_per_split;
+        const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
+        if (!wait_bounded(tmem_empty, acc_phase ^ 1u, abort_flag, kFaultMma)) {
+          aborted = true;
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kt = k0; kt < k1; ++kt) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma) ||
+              !wait_bounded(&sf_full[sf_buf], sf_phase, abort_flag, kFaultMma)) {
+            aborted = true;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sa = smem_base + stage * C::STAGE_BYTES;
+          const uint32_t sb = sa + C::A_BYTES;
+          const uint32_t tsfa = tmem + SF_COL + sf_buf * SF_BUF_COLS;
+          const uint32_t tsfb = tsfa + 16u;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t adesc = ptx::smem_desc(sa + 32u * j, 16, 1024, 2);
+            const uint64_t bdesc = ptx::smem_desc(sb + 32u * j, 16, 1024, 2);
+            ptx::tc_mma_nvf4(tmem, adesc, bdesc, C::IDESC, tsfa + 4u * j, tsfb + C::SFB_COLS * j,
+                             (kt != k0 || j != 0) ? 1u : 0u);
+          }
+          ptx::tc_commit(&empty[stage]);
+          ptx::tc_commit(&sf_empty[sf_buf]);
+          if (++sf_buf == NSF) {
+            sf_buf = 0;
+            sf_phase ^= 1u;
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (aborted) break;
+        ptx::tc_commit(tmem_full);
+        acc_phase ^= 1u;
+      }
+      if (aborted) {
+        ptx::tc_commit(drain);
+        drain_wait(drain, 0);
+      }
+    }
+  } else if (warp < EPI_WARP0) {
+    // ----------------------------------------------------- scale-copy warps --
+    if (lane == 0) {
+      const int part = warp - SF_WARP0;  // 0: weight scales, 1: token scales
+      const uint32_t smem_base = ptx::smem_u32(smem);
+      uint32_t stage = 0, phase = 0, sf_buf = 0, sf_phase = 0;
+      bool aborted = false;
+      for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
+        const int sp = u / p.num_w_tiles;
+        const int k0 = sp * p.k_tiles_per_split;
+        const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
+        for (int kt = k0; kt < k1; ++kt) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales) ||
+              !wait_bounded(&sf_empty[sf_buf], sf_phase ^ 1u, abort_flag, kFaultScales)) {
+            aborted = true;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t ssfa = smem_base + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
+          const uint32_t ssfb = ssfa + C::SFA_BYTES;
+          const uint32_t tsfa = tmem + SF_COL + sf_buf * SF_BUF_COLS;
+          const uint32_t tsfb = tsfa + 16u;
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if (part == 0) {
+              ptx::tc_cp_32x128b_warpx4(tsfa + 4u * j, ptx::smem_desc(ssfa + 512u * j, 0, 128, 0));
+            } else {
+#pragma unroll
+              for (int h = 0; h < C::SFB_BLOCKS; ++h)
+                ptx::tc_cp_32x128b_warpx4(tsfb + C::SFB_COLS * j + 4u * h,
+                                          ptx::smem_desc(ssfb + 2048u * h + 512u * j, 0, 128, 0));
+            }
+          }
+          ptx::tc_commit(&sf_full[sf_buf]);
+          if (++sf_buf == NSF) {
+            sf_buf = 0;
+            sf_phase ^= 1u;
+          }
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (aborted) {
+        ptx::tc_commit(drain_sf);
+        drain_wait(drain_sf, 0);
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue --
+    const int q = warp & 3;  // tensor-memory lane quarter (warps 4..7 -> 0..3)
+    const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
+    uint32_t acc_phase = 0;
+    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
+      const int wt = u % p.num_w_tiles;
+      if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue)) break;
+      ptx::tc_fence_after();
+      const int n = wt * BW + q * 32 + lane;   // this thread's output column
+      const bool n_ok = n < p.N;
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+#pragma unroll
+      for (int c0 = 0; c0 < BNT; c0 += 32) {
+        uint32_t r[32];
+        if (BNT >= 32) {
+          ptx::tc_ld_32x32b_x32(lane_base + c0, r);
+        } else {
+          tc_ld_32x32b_x16(lane_base + c0, r);
+        }
+        ptx::tc_wait_ld();
+        const int cols = BNT < 32 ? BNT : 32;
+#pragma unroll
+        for (int i = 0; i < cols; ++i) {
+          const int m = c0 + i;                 // token
+          if (m >= p.M || !n_ok) continue;
+          const float v = __uint_as_float(r[i]) * alpha;
+          if (p.partial != nullptr) {
+            red_add_f32(p.partial + static_cast<int64_t>(m) * p.N + n, v);
+          } else if (p.y_fp32) {
+            reinterpret_cast<float*>(p.y)[static_cast<int64_t>(m) * p.ldy + n] = v;
+          } else {
+            reinterpret_cast<__nv_bfloat16*>(p.y)[static_cast<int64_t>(m) * p.ldy + n] =
+                __float2bfloat16_rn(v);
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(tmem_empty);
+      acc_phase ^= 1u;
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Split mode: Y = the FP32 sums (already scaled by 1/(g_a g_b)), converted.
+__global__ void __launch_bounds__(256)
+    finalize_kernel(const float* __restrict__ partial, int64_t m, int64_t n, void* y,
+                    int64_t ldy, int y_fp32) {
+  const int64_t total = m * n;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / n, c = i - r * n;
+    const float v = partial[i];
+    if (y_fp32)
+      reinterpret_cast<float*>(y)[r * ldy + c] = v;
+    else
+      reinterpret_cast<__nv_bfloat16*>(y)[r * ldy + c] = __float2bfloat16_rn(v);
+  }
+}
+
+}  // namespace skinny
+}  // namespace nvfp4

@@ -37,6 +37,14 @@
 //           by the TMA unit). Per-thread 16-byte stores of whole rows would
 //           cost one L2 sector write each and steal L2 bandwidth from the
 //           operand loads.
+// Fused SwiGLU mode (gate_up projection of a gated MLP): the weight rows are
+// interleaved in blocks of 128 — gate rows of block b, then up rows of block
+// b — so a 256-column tile holds 128 gate and the matching 128 up columns.
+// The epilogue then forms h = silu(gate) * up with exactly the roundings of
+// the unfused path (gate/up rounded to bf16 as the GEMM stores them, the same
+// SwiGLU expression, h rounded to bf16) and quantizes h to NVFP4 with a
+// calibrated static global using the quantizer's arithmetic, writing codes
+// and swizzled scales of h instead of the 2*ffn-wide bf16 output.
 // Every mbarrier wait is bounded in time; on expiry the kernel records a fault
 // word, both CTAs of the pair stop, in-flight copies and MMAs are drained
 // (again with a bound) and tensor memory is released before the CTAs exit.
@@ -45,13 +53,12 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include "fault.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
+#include "silu_mul.cuh"
 
 namespace nvfp4 {
-
-// Nonzero after a bounded wait expired in any kernel; read and cleared by
-// nvfp4_read_fault. Bits name the role that gave up.
-__device__ unsigned int g_fault_word;
 
 namespace gemm {
 
@@ -81,7 +88,8 @@ constexpr int EPI_CHUNK_BYTES = 32 * 64;      // 32 rows x 64 bytes, 64-byte swi
 constexpr int EPI_WARP_BYTES = 2 * EPI_CHUNK_BYTES;
 constexpr int EPI_OFF = STAGES * STAGE_BYTES;  // staging tiles after the ring
 constexpr int BAR_OFF = EPI_OFF + NUM_EPI_WARPS * EPI_WARP_BYTES;
-constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(BAR_OFF) + 512;
+constexpr int RTAB_OFF = BAR_OFF + 512;      // fused mode: g_h / dec(s) for 128 codes
+constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(RTAB_OFF) + 512;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr uint64_t kDrainLimitNs = 100000000ull;  // 0.1 s for the abort drain
 
@@ -101,6 +109,13 @@ struct Params {
   void* y;
   int64_t ldy;
   int y_fp32;
+  // fused SwiGLU + quantize mode (y unused): h = [M][ffn], ffn = N / 2
+  int fused;
+  const float* h_global;   // static global of h
+  uint8_t* h_codes;        // [M][ffn/2]
+  uint8_t* h_sf;           // swizzled scales of [M][ffn]
+  int64_t h_atoms;         // 512-byte atoms per 128-row block = ffn / 64
+  int m_pad;               // rows of the scale buffer = ceil(M/128)*128
 };
 
 // Band rasterization: consecutive tiles walk GROUP_M M-tiles down one N band,
@@ -188,6 +203,33 @@ __device__ __forceinline__ void stage_f32(uint32_t chunk, int row, const uint32_
                       __float_as_uint(__uint_as_float(r[off + 4 * u + 3]) * alpha));
 }
 
+// One 16-column block of h for the fused mode: gate/up accumulators ->
+// bf16 (as stored by the plain GEMM) -> SwiGLU -> bf16 h -> NVFP4 codes with
+// the quantizer's rounding. Returns the block's E4M3 scale; codes in w[0..1].
+__device__ __forceinline__ uint32_t swiglu_quant_block(const uint32_t* g, const uint32_t* u,
+                                                       float alpha, float gh, const float* rtab,
+                                                       uint32_t& w0, uint32_t& w1) {
+  float hv[16];
+  float amax = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float gb = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[i]) * alpha));
+    const float ub = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[i]) * alpha));
+    hv[i] = __bfloat162float(__float2bfloat16_rn(act::swiglu(gb, ub)));
+    amax = fmaxf(amax, fabsf(hv[i]));
+  }
+  const uint32_t sc = ptx::cvt_e4m3(__fmul_rn(quant::div6_rn(amax), gh));
+  const float r = rtab[sc];
+  float f[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(hv[i], r);
+  w0 = ptx::cvt_e2m1x8(f);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) f[i] = __fmul_rn(hv[8 + i], r);
+  w1 = ptx::cvt_e2m1x8(f);
+  return sc;
+}
+
 // Tensor-memory columns of scale buffer `buf`: A's 16, then B's 32.
 __device__ __forceinline__ uint32_t sfa_cols(uint32_t tmem, uint32_t buf) {
   return tmem + SF_COL + buf * SF_BUF_COLS;
@@ -268,7 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::tma_prefetch_desc(&tmB);
     ptx::tma_prefetch_desc(&tmSFA);
     ptx::tma_prefetch_desc(&tmSFB);
-    ptx::tma_prefetch_desc(&tmY);
+    if (!p.fused) ptx::tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -409,6 +451,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue --
+    float* rtab = reinterpret_cast<float*>(smem + RTAB_OFF);
+    if (p.fused) {
+      // E4M3 code -> g_h / dec(code), as the quantizer tabulates it
+      const float gh = __ldg(p.h_global);
+      const int t = threadIdx.x - EPI_WARP0 * 32;
+      if (t < 128) {
+        const float ds = ptx::e4m3_value(static_cast<uint32_t>(t));
+        rtab[t] = (ds == 0.0f) ? 0.0f : __fdiv_rn(gh, ds);
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * NUM_EPI_WARPS) : "memory");
+    }
     const int q = warp & 3;                     // tensor-memory lane quarter
     const int half = (warp - EPI_WARP0) >> 2;   // accumulator columns [128*half, +128)
     const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
@@ -436,6 +489,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tile_coords(t, p, mb, nb);
       if (!wait_bounded(tmem_full, acc_phase, ab, kFaultEpilogue)) break;
       ptx::tc_fence_after();
+      if (p.fused) {
+        // gate columns [64 half, +64) and the matching up columns (+128)
+        uint32_t g0[32], g1[32], u0[32], u1[32];
+        const uint32_t lb = tmem + (static_cast<uint32_t>(q * 32) << 16) + 64u * half;
+        ptx::tc_ld_32x32b_x32(lb + 0u, g0);
+        ptx::tc_ld_32x32b_x32(lb + 32u, g1);
+        ptx::tc_ld_32x32b_x32(lb + 128u, u0);
+        ptx::tc_ld_32x32b_x32(lb + 160u, u1);
+        ptx::tc_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(release);
+        acc_phase ^= 1u;
+        const int row = mb * BM + static_cast<int>(rank) * HALF + q * 32 + lane;
+        if (row >= p.m_pad) continue;  // no scale bytes past the padded rows
+        const float gh = __ldg(p.h_global);
+        const int hc0 = nb * 128 + 64 * half;  // first h column of this thread
+        uint32_t c[8];
+        uint32_t sfw = swiglu_quant_block(g0, u0, alpha, gh, rtab, c[0], c[1]);
+        sfw |= swiglu_quant_block(g0 + 16, u0 + 16, alpha, gh, rtab, c[2], c[3]) << 8;
+        sfw |= swiglu_quant_block(g1, u1, alpha, gh, rtab, c[4], c[5]) << 16;
+        sfw |= swiglu_quant_block(g1 + 16, u1 + 16, alpha, gh, rtab, c[6], c[7]) << 24;
+        // rows in [M, m_pad) were zero-filled operands: h = 0, scales 0
+        if (row < p.M) {
+          uint4* dst = reinterpret_cast<uint4*>(p.h_codes + static_cast<int64_t>(row) * (p.N / 4) +
+                                                hc0 / 2);
+          dst[0] = make_uint4(c[0], c[1], c[2], c[3]);
+          dst[1] = make_uint4(c[4], c[5], c[6], c[7]);
+        }
+        *reinterpret_cast<uint32_t*>(
+            p.h_sf + ((row >> 7) * p.h_atoms + (hc0 >> 6)) * 512 + (row & 31) * 16 +
+            ((row & 127) >> 5) * 4) = sfw;
+        continue;
+      }
       uint32_t r0[32], r1[32], r2[32], r3[32];
       const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + ACC_COL + half * 128u;
       ptx::tc_ld_32x32b_x32(taddr + 0u, r0);

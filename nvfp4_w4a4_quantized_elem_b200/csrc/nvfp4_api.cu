@@ -16,6 +16,7 @@
 
 #include "fold.cuh"
 #include "gemm_sm100.cuh"
+#include "gemm_skinny.cuh"
 #include "quant.cuh"
 #include "silu_mul.cuh"
 
@@ -26,6 +27,7 @@ constexpr int kMaxDevices = 64;
 struct DeviceState {
   int sms = 0;
   bool gemm_smem_set = false;
+  unsigned skinny_smem_set = 0;       // bit per token-tile instantiation
   float* noalloc_partials = nullptr;  // device address of g_noalloc_partials
 };
 
@@ -77,6 +79,21 @@ nvfp4_status launch_status() {
 }
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// CTAs of the amax pass: enough that every thread streams ~8 16-byte chunks
+// (the contiguous path is flat over elements, the strided one a warp per
+// row), at most 2 per SM. Sizing by rows alone starved few-row inputs.
+int64_t amax_blocks(int64_t rows, int64_t k, int64_t ldx, int sms) {
+  using namespace nvfp4::quant;
+  const int64_t per_block = (ldx == k) ? static_cast<int64_t>(kAmaxThreads) * 8 * 8
+                                       : static_cast<int64_t>(kAmaxThreads / 32);
+  const int64_t units = (ldx == k) ? rows * k : rows;
+  int64_t blocks = ceil_div(units, per_block);
+  const int64_t cap = static_cast<int64_t>(sms) * kAmaxBlocksPerSM;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return blocks;
+}
 
 // Scratch of nvfp4_quantize_noalloc: the amax pass's per-CTA partial maxima.
 // Host code must not use this name as a pointer (it is a host-side stand-in);
@@ -150,9 +167,7 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
 
   int nparts = 0;
   if (dynamic) {
-    const int64_t warps_per_block = kAmaxThreads / 32;
-    int64_t blocks = ceil_div(rows, warps_per_block);
-    if (blocks > static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM) blocks = static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM;
+    int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
     if (blocks > kMaxPartials) blocks = kMaxPartials;
     if (blocks < 1) blocks = 1;
     nparts = static_cast<int>(blocks);
@@ -200,10 +215,7 @@ nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k, int6
 
   int nparts = 0;
   if (global_in == nullptr) {
-    int64_t blocks = ceil_div(rows, kAmaxThreads / 32);
-    if (blocks > static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM)
-      blocks = static_cast<int64_t>(st->sms) * kAmaxBlocksPerSM;
-    if (blocks < 1) blocks = 1;
+    const int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
     if (blocks > NVFP4_NOALLOC_MAX_PARTIALS) return NVFP4_ERR_UNSUPPORTED;
     nparts = static_cast<int>(blocks);
     amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
@@ -230,12 +242,41 @@ nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k, int6
   return launch_status();
 }
 
-size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
-  (void)m;
-  (void)n;
-  (void)k;
-  return 0;
+nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k, int64_t ldx,
+                                    float* running_amax, float* global_out, void* workspace,
+                                    size_t workspace_bytes, nvfp4_stream_t stream) {
+  using namespace nvfp4::quant;
+  if (rows < 0 || k <= 0 || running_amax == nullptr || global_out == nullptr || ldx < k)
+    return NVFP4_ERR_INVALID_ARG;
+  if (k % 16 != 0) return NVFP4_ERR_UNSUPPORTED;
+  if (rows > 0 && x == nullptr) return NVFP4_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < nvfp4_quantize_workspace_bytes(rows, k))
+    return NVFP4_ERR_INVALID_ARG;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(workspace, 16) || !aligned(running_amax, 4) ||
+      !aligned(global_out, 4))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
+  if (blocks > kMaxPartials) blocks = kMaxPartials;
+  amax_kernel<<<static_cast<unsigned>(blocks), kAmaxThreads, 0, s>>>(
+      static_cast<const uint16_t*>(x), rows, k, ldx, static_cast<float*>(workspace));
+  if (nvfp4_status e = launch_status()) return e;
+  calibrate_kernel<<<1, 256, 0, s>>>(static_cast<const float*>(workspace),
+                                     static_cast<int>(blocks), running_amax, global_out);
+  return launch_status();
 }
+
+size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+  (void)k;
+  if (m < 1 || n < 1) return 0;
+  // few-token GEMMs split K across CTAs and sum FP32 partials of Y here
+  return m <= 64 ? static_cast<size_t>(m) * static_cast<size_t>(n) * sizeof(float) : 0;
+}
+
+}  // extern "C"
 
 namespace {
 
@@ -282,15 +323,164 @@ nvfp4_status encode_sf(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
+template <int BNT>
+nvfp4_status launch_skinny(DeviceState* st, int bit, const CUtensorMap& tmW, const CUtensorMap& tmX,
+                           const CUtensorMap& tmSFW, const CUtensorMap& tmSFX,
+                           const nvfp4::skinny::Params& p, int grid, cudaStream_t s) {
+  using nvfp4::skinny::Cfg;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!(st->skinny_smem_set & (1u << bit))) {
+      if (cudaFuncSetAttribute(nvfp4::skinny::skinny_kernel<BNT>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(Cfg<BNT>::SMEM_BYTES)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+      }
+      st->skinny_smem_set |= 1u << bit;
+    }
+  }
+  nvfp4::skinny::skinny_kernel<BNT><<<grid, nvfp4::skinny::NUM_THREADS, Cfg<BNT>::SMEM_BYTES, s>>>(
+      tmW, tmX, tmSFW, tmSFX, p);
+  return launch_status();
+}
+
+// Few tokens (m <= 64): Y^T = B A^T with the weights on the MMA's 128-row
+// side and the tokens as its N; K split across CTAs when the weight tiles
+// cannot fill the GPU and a workspace for the FP32 partial sums is given.
+nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
+                         const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
+                         void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
+                         void* workspace, size_t workspace_bytes, cudaStream_t s) {
+  using namespace nvfp4::skinny;
+  const int bnt = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
+  CUtensorMap tmW, tmX, tmSFW, tmSFX;
+  if (nvfp4_status e = encode_2d(enc, &tmW, b_codes, static_cast<uint64_t>(k / 2),
+                                 static_cast<uint64_t>(n), BW))
+    return e;
+  if (nvfp4_status e = encode_2d(enc, &tmX, a_codes, static_cast<uint64_t>(k / 2),
+                                 static_cast<uint64_t>(m), static_cast<uint32_t>(bnt)))
+    return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFW, b_sf, n, k, 1u)) return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFX, a_sf, m, k, bnt > 128 ? 2u : 1u)) return e;
+  Params p;
+  p.M = static_cast<int>(m);
+  p.N = static_cast<int>(n);
+  p.K = static_cast<int>(k);
+  p.num_w_tiles = static_cast<int>(ceil_div(n, BW));
+  p.num_k_tiles = static_cast<int>(ceil_div(k, BK));
+  p.a_global = a_global;
+  p.b_global = b_global;
+  p.y = y;
+  p.ldy = ldy;
+  p.y_fp32 = y_dtype;
+  p.partial = nullptr;
+  int splits = 1;
+  const size_t need = static_cast<size_t>(m) * static_cast<size_t>(n) * sizeof(float);
+  if (workspace != nullptr && workspace_bytes >= need && aligned(workspace, 16)) {
+    splits = st->sms / p.num_w_tiles;
+    if (splits > p.num_k_tiles) splits = p.num_k_tiles;
+    if (splits < 1) splits = 1;
+  }
+  p.k_tiles_per_split = static_cast<int>(ceil_div(p.num_k_tiles, splits));
+  splits = static_cast<int>(ceil_div(p.num_k_tiles, p.k_tiles_per_split));  // no empty slice
+  p.splits = splits;
+  if (splits > 1) {
+    p.partial = static_cast<float*>(workspace);
+    if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+  }
+  const int64_t units = static_cast<int64_t>(p.num_w_tiles) * splits;
+  const int grid = static_cast<int>(units < st->sms ? units : st->sms);
+  nvfp4_status e;
+  switch (bnt) {
+    case 16: e = launch_skinny<16>(st, 0, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    case 32: e = launch_skinny<32>(st, 1, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    case 64: e = launch_skinny<64>(st, 2, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    case 128: e = launch_skinny<128>(st, 3, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    default: e = launch_skinny<256>(st, 4, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+  }
+  if (e != NVFP4_OK || splits == 1) return e;
+  int64_t blocks = ceil_div(m * n, 256);
+  if (blocks > static_cast<int64_t>(st->sms) * 8) blocks = static_cast<int64_t>(st->sms) * 8;
+  finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
+      static_cast<const float*>(workspace), m, n, y, ldy, y_dtype);
+  return launch_status();
+}
+
+// The paired-CTA kernel (cta_group::2, 256x256 tiles): M, N, K, tile counts
+// and tensor maps filled in here; output / fused fields come in `p`.
+nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
+                         const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes,
+                         const uint8_t* b_sf, int64_t m, int64_t n, int64_t k,
+                         nvfp4::gemm::Params p, cudaStream_t stream) {
+  using namespace nvfp4::gemm;
+  CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+  std::memset(&tmY, 0, sizeof tmY);
+  if (nvfp4_status e = encode_2d(enc, &tmA, a_codes, static_cast<uint64_t>(k / 2),
+                                 static_cast<uint64_t>(m), HALF))
+    return e;
+  if (nvfp4_status e = encode_2d(enc, &tmB, b_codes, static_cast<uint64_t>(k / 2),
+                                 static_cast<uint64_t>(n), HALF))
+    return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFA, a_sf, m, k, 1u)) return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFB, b_sf, n, k, 2u)) return e;
+  if (!p.fused)
+    if (nvfp4_status e = encode_y(enc, &tmY, p.y, m, n, p.ldy, p.y_fp32)) return e;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (!st->gemm_smem_set) {
+      if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(SMEM_BYTES)) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+      }
+      st->gemm_smem_set = true;
+    }
+  }
+  p.M = static_cast<int>(m);
+  p.N = static_cast<int>(n);
+  p.K = static_cast<int>(k);
+  p.num_m_blk = static_cast<int>(ceil_div(m, BM));
+  p.num_n_blk = static_cast<int>(ceil_div(n, BN));
+  p.num_k_tiles = static_cast<int>(ceil_div(k, BK));
+  const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
+  if (tiles >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;
+  // one CTA pair (cluster of 2 SMs) per 256x256 tile at a time, persistent
+  const int64_t max_pairs = st->sms / 2;
+  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
+  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmSFA, tmSFB, tmY, p) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return launch_status();
+}
+
 }  // namespace
+
+extern "C" {
 
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
                         void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
                         void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
   using namespace nvfp4::gemm;
-  (void)workspace;
-  (void)workspace_bytes;
   if (!a_codes || !a_sf || !a_global || !b_codes || !b_sf || !b_global || !y)
     return NVFP4_ERR_INVALID_ARG;
   if (m < 1 || n < 1 || k < 1 || (y_dtype != 0 && y_dtype != 1) || ldy < n)
@@ -307,64 +497,54 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   if (nvfp4_status e = current_device(&dev, &st)) return e;
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (nvfp4_status e = get_encoder(&enc)) return e;
+  if (m <= 64)
+    return gemm_skinny(enc, st, a_codes, a_sf, a_global, b_codes, b_sf, b_global, y, y_dtype, ldy,
+                       m, n, k, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
 
-  CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
-  if (nvfp4_status e = encode_2d(enc, &tmA, a_codes, static_cast<uint64_t>(k / 2),
-                                 static_cast<uint64_t>(m), HALF))
-    return e;
-  if (nvfp4_status e = encode_2d(enc, &tmB, b_codes, static_cast<uint64_t>(k / 2),
-                                 static_cast<uint64_t>(n), HALF))
-    return e;
-  if (nvfp4_status e = encode_sf(enc, &tmSFA, a_sf, m, k, 1u)) return e;
-  if (nvfp4_status e = encode_sf(enc, &tmSFB, b_sf, n, k, 2u)) return e;
-  if (nvfp4_status e = encode_y(enc, &tmY, y, m, n, ldy, y_dtype)) return e;
-
-  {
-    std::lock_guard<std::mutex> lock(g_mutex);
-    if (!st->gemm_smem_set) {
-      if (cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(SMEM_BYTES)) != cudaSuccess) {
-        cudaGetLastError();
-        return NVFP4_ERR_CUDA;
-      }
-      st->gemm_smem_set = true;
-    }
-  }
-  Params p;
-  p.M = static_cast<int>(m);
-  p.N = static_cast<int>(n);
-  p.K = static_cast<int>(k);
-  p.num_m_blk = static_cast<int>(ceil_div(m, BM));
-  p.num_n_blk = static_cast<int>(ceil_div(n, BN));
-  p.num_k_tiles = static_cast<int>(ceil_div(k, BK));
+  nvfp4::gemm::Params p;
+  std::memset(&p, 0, sizeof p);
   p.a_global = a_global;
   p.b_global = b_global;
   p.y = y;
   p.ldy = ldy;
   p.y_fp32 = y_dtype;
-  const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
-  if (tiles >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;
-  // one CTA pair (cluster of 2 SMs) per 256x256 tile at a time, persistent
-  const int64_t max_pairs = st->sms / 2;
-  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmSFA, tmSFB, tmY, p) != cudaSuccess) {
-    cudaGetLastError();
-    return NVFP4_ERR_CUDA;
-  }
-  return launch_status();
+  return gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, n, k, p,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf,
+                                     const float* a_global, const uint8_t* b_codes,
+                                     const uint8_t* b_sf, const float* b_global,
+                                     const float* h_global, uint8_t* h_codes, uint8_t* h_sf,
+                                     int64_t m, int64_t ffn, int64_t k, nvfp4_stream_t stream) {
+  if (!a_codes || !a_sf || !a_global || !b_codes || !b_sf || !b_global || !h_global ||
+      !h_codes || !h_sf)
+    return NVFP4_ERR_INVALID_ARG;
+  if (m < 1 || ffn < 1 || k < 1) return NVFP4_ERR_INVALID_ARG;
+  if (ffn % 128 != 0 || k % 32 != 0 || m >= (int64_t{1} << 31) || 2 * ffn >= (int64_t{1} << 31) ||
+      k >= (int64_t{1} << 31))
+    return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
+      !aligned(h_codes, 16) || !aligned(h_sf, 16) || !aligned(a_global, 4) ||
+      !aligned(b_global, 4) || !aligned(h_global, 4))
+    return NVFP4_ERR_MISALIGNED;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (nvfp4_status e = get_encoder(&enc)) return e;
+  nvfp4::gemm::Params p;
+  std::memset(&p, 0, sizeof p);
+  p.a_global = a_global;
+  p.b_global = b_global;
+  p.fused = 1;
+  p.h_global = h_global;
+  p.h_codes = h_codes;
+  p.h_sf = h_sf;
+  p.h_atoms = ffn / 64;
+  p.m_pad = static_cast<int>(ceil_div(m, 128) * 128);
+  return gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, 2 * ffn, k, p,
+                     reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status nvfp4_fuse_group_scales(int n_modules, const int64_t* rows_per_module, int64_t k,

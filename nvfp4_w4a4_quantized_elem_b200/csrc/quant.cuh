@@ -221,5 +221,26 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
   }
 }
 
+// Calibration step: running_amax = max(running_amax, max of the partials);
+// global_out = 2688 / running_amax (1 when that is 0 or not finite). One CTA.
+__global__ void __launch_bounds__(256)
+    calibrate_kernel(const float* __restrict__ partials, int nparts, float* running_amax,
+                     float* global_out) {
+  __shared__ uint32_t s_red[8];
+  uint32_t m = 0;
+  for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, __float_as_uint(partials[i]));
+  m = __reduce_max_sync(0xFFFFFFFFu, m);
+  if ((threadIdx.x & 31) == 0) s_red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < 8; ++w) m = max(m, s_red[w]);
+    const float amax = fmaxf(*running_amax, __uint_as_float(m));
+    *running_amax = amax;
+    float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, amax);
+    if (!isfinite(g)) g = 1.0f;
+    *global_out = g;
+  }
+}
+
 }  // namespace quant
 }  // namespace nvfp4

@@ -13,6 +13,12 @@ namespace act {
 
 constexpr int kThreads = 256;
 
+// silu(g) * u in FP32 with explicitly rounded steps, shared by the
+// standalone kernel and the fused GEMM epilogue so both give the same bits.
+__device__ __forceinline__ float swiglu(float g, float u) {
+  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+}
+
 // h = bf16(silu(gate) * up), gate = y[:, :n], up = y[:, n:2n]; one warp per
 // row, 16-byte vectors (8 elements) per lane.
 __global__ void __launch_bounds__(kThreads)
@@ -35,8 +41,8 @@ __global__ void __launch_bounds__(kThreads)
       for (int e = 0; e < 4; ++e) {
         const float g0 = __uint_as_float(gw[e] << 16), g1 = __uint_as_float(gw[e] & 0xFFFF0000u);
         const float u0 = __uint_as_float(uw[e] << 16), u1 = __uint_as_float(uw[e] & 0xFFFF0000u);
-        const float h0 = g0 / (1.0f + expf(-g0)) * u0;
-        const float h1 = g1 / (1.0f + expf(-g1)) * u1;
+        const float h0 = swiglu(g0, u0);
+        const float h1 = swiglu(g1, u1);
         const __nv_bfloat162 p = __floats2bfloat162_rn(h0, h1);
         ow[e] = *reinterpret_cast<const uint32_t*>(&p);
       }

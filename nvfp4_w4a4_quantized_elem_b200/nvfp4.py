@@ -24,7 +24,8 @@ STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPO
 
 # every symbol include/nvfp4.h declares
 EXPORTS = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_quantize_workspace_bytes",
-           "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_gemm_workspace_bytes", "nvfp4_gemm",
+           "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_calibrate_global",
+           "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_gemm_swiglu_quant",
            "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault")
 
 _lib = None
@@ -56,8 +57,10 @@ def lib() -> ctypes.CDLL:
             "nvfp4_quantize_workspace_bytes": (SZ, [I64, I64]),
             "nvfp4_quantize": (I, [P, I64, I64, I64, P, P, P, P, P, SZ, P]),
             "nvfp4_quantize_noalloc": (I, [P, I64, I64, I64, P, P, P, P, P]),
+            "nvfp4_calibrate_global": (I, [P, I64, I64, I64, P, P, P, SZ, P]),
             "nvfp4_gemm_workspace_bytes": (SZ, [I64, I64, I64]),
             "nvfp4_gemm": (I, [P, P, P, P, P, P, P, I, I64, I64, I64, I64, P, SZ, P]),
+            "nvfp4_gemm_swiglu_quant": (I, [P, P, P, P, P, P, P, P, P, I64, I64, I64, P]),
             "nvfp4_fuse_group_scales": (I, [I, P, I64, P, P, P, P, P]),
             "nvfp4_silu_mul": (I, [P, I64, I64, I64, P, I64, P]),
             "nvfp4_read_fault": (I, [P, U32P]),
@@ -155,11 +158,41 @@ def quantize_noalloc(x: torch.Tensor, out: NVFP4Tensor, global_scale: torch.Tens
     return out
 
 
+class Calibrator:
+    """Static global scale from a stream of calibration batches
+    (nvfp4_calibrate_global): observe() each batch, then use .global_scale
+    as quantize(..., global_scale=...)."""
+
+    def __init__(self, device="cuda"):
+        self.running_amax = torch.zeros(1, dtype=torch.float32, device=device)
+        self.global_scale = torch.ones(1, dtype=torch.float32, device=device)
+        self._ws = None
+
+    def observe(self, x: torch.Tensor, stream: torch.cuda.Stream | None = None) -> torch.Tensor:
+        _require_cuda(x, "x", torch.bfloat16)
+        if x.dim() != 2 or x.stride(1) != 1:
+            raise ValueError("x must be 2-D with unit stride along k")
+        rows, k = x.shape
+        need = quantize_workspace_bytes(rows, k)
+        if self._ws is None or self._ws.numel() < need:
+            self._ws = torch.empty(need, dtype=torch.uint8, device=x.device)
+        st = lib().nvfp4_calibrate_global(_ptr(x), rows, k, x.stride(0), _ptr(self.running_amax),
+                                          _ptr(self.global_scale), _ptr(self._ws), self._ws.numel(),
+                                          _stream(stream))
+        _check(st, "nvfp4_calibrate_global")
+        return self.global_scale
+
+
+def gemm_workspace_bytes(m: int, n: int, k: int) -> int:
+    return int(lib().nvfp4_gemm_workspace_bytes(m, n, k))
+
+
 def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out: torch.Tensor | None = None,
-         out_dtype: torch.dtype = torch.bfloat16,
+         out_dtype: torch.dtype = torch.bfloat16, workspace: torch.Tensor | None = None,
          stream: torch.cuda.Stream | None = None) -> torch.Tensor:
     """nvfp4_gemm: Y[m, n] = dequant(A) @ dequant(B).T (A = activations
-    [m, k], B = weights [n, k]); bf16 or fp32 output."""
+    [m, k], B = weights [n, k]); bf16 or fp32 output. ``workspace`` (at least
+    gemm_workspace_bytes) lets few-token GEMMs split K across the GPU."""
     if a.k != b.k:
         raise ValueError("k mismatch")
     m, n, k = a.rows, b.rows, a.k
@@ -168,10 +201,44 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out: torch.Tensor | None = None,
     if out.dtype not in (torch.bfloat16, torch.float32) or out.stride(1) != 1:
         raise ValueError("out must be bf16/fp32 with unit column stride")
     y_dtype = 0 if out.dtype == torch.bfloat16 else 1
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     st = lib().nvfp4_gemm(_ptr(a.codes), _ptr(a.sf), _ptr(a.global_scale),
                           _ptr(b.codes), _ptr(b.sf), _ptr(b.global_scale),
-                          _ptr(out), y_dtype, out.stride(0), m, n, k, None, 0, _stream(stream))
+                          _ptr(out), y_dtype, out.stride(0), m, n, k, _ptr(workspace), ws_bytes,
+                          _stream(stream))
     _check(st, "nvfp4_gemm")
+    return out
+
+
+def interleave_gate_up(w_gate_up: torch.Tensor) -> torch.Tensor:
+    """Row order nvfp4_gemm_swiglu_quant expects: [2*ffn, k] with gate rows
+    [0, ffn) and up rows [ffn, 2ffn) -> blocks of 128 (gate b, up b, ...).
+    Offline weight preparation (a row permutation)."""
+    two_ffn = w_gate_up.shape[0]
+    ffn = two_ffn // 2
+    if two_ffn % 256:
+        raise ValueError("ffn must be a multiple of 128")
+    idx = torch.arange(two_ffn, device=w_gate_up.device).view(2, ffn // 128, 128)
+    return w_gate_up[idx.transpose(0, 1).reshape(-1)]
+
+
+def gemm_swiglu_quant(a: NVFP4Tensor, b_interleaved: NVFP4Tensor, h_global: torch.Tensor,
+                      out: NVFP4Tensor | None = None,
+                      stream: torch.cuda.Stream | None = None) -> NVFP4Tensor:
+    """nvfp4_gemm_swiglu_quant: NVFP4 h = quantize(silu(gate) * up, h_global)
+    straight from the gate_up GEMM (weights row-interleaved, see
+    interleave_gate_up)."""
+    if a.k != b_interleaved.k:
+        raise ValueError("k mismatch")
+    m, ffn, k = a.rows, b_interleaved.rows // 2, a.k
+    if out is None:
+        out = NVFP4Tensor.empty(m, ffn, a.codes.device)
+    out.global_scale.copy_(h_global.reshape(1))
+    st = lib().nvfp4_gemm_swiglu_quant(_ptr(a.codes), _ptr(a.sf), _ptr(a.global_scale),
+                                       _ptr(b_interleaved.codes), _ptr(b_interleaved.sf),
+                                       _ptr(b_interleaved.global_scale), _ptr(h_global),
+                                       _ptr(out.codes), _ptr(out.sf), m, ffn, k, _stream(stream))
+    _check(st, "nvfp4_gemm_swiglu_quant")
     return out
 
 

@@ -119,3 +119,25 @@ def test_silu_argument_checks(L):
     assert f(P(FAKE), 4, 12, 24, P(FAKE), 16, None) == UNSUPPORTED  # n % 8
     assert f(P(FAKE), 4, 16, 16, P(FAKE), 16, None) == INVALID      # ldy < 2n
     assert f(P(FAKE + 2), 4, 16, 32, P(FAKE), 16, None) == MISALIGNED
+
+
+def test_interleave_gate_up_permutation():
+    import torch
+    from nvfp4_w4a4_quantized_elem_b200 import nvfp4
+    ffn, k = 384, 4
+    w = torch.arange(2 * ffn, dtype=torch.float32)[:, None].expand(2 * ffn, k).contiguous()
+    wi = nvfp4.interleave_gate_up(w)[:, 0].long()
+    for b in range(ffn // 128):
+        assert torch.equal(wi[256 * b:256 * b + 128], torch.arange(128 * b, 128 * b + 128))
+        assert torch.equal(wi[256 * b + 128:256 * b + 256],
+                           torch.arange(ffn + 128 * b, ffn + 128 * b + 128))
+
+
+def test_swiglu_quant_argument_checks(L):
+    f = L.nvfp4_gemm_swiglu_quant
+    args = lambda ffn=256, k=512, h=FAKE: (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE),
+                                           P(FAKE), P(h), P(FAKE), 8, ffn, k, None)
+    assert f(*args(ffn=200)) == UNSUPPORTED      # ffn % 128
+    assert f(*args(k=48)) == UNSUPPORTED
+    assert f(*args(h=FAKE + 8)) == MISALIGNED
+    assert f(*args(h=None)) == INVALID

@@ -24,19 +24,30 @@ def gaussian(rows, k, seed, sigma=1.0):
     return (torch.randn((rows, k), generator=g) * sigma).to(torch.bfloat16)
 
 
-def run_case(nv, orc, x, w, dtypes=(torch.bfloat16, torch.float32), what=""):
+def run_case(nv, orc, x, w, dtypes=(torch.bfloat16, torch.float32), what="",
+             workspaces=(False, True)):
+    """Both output dtypes; with and without a GEMM workspace (few-token GEMMs
+    split K across CTAs only when one is given)."""
     qa, qb = orc.quantize(bits(x)), orc.quantize(bits(w))
     ref = orc.gemm(qa, qb)
     rn, cn = norms(orc, qa), norms(orc, qb)
     A, B = upload(qa), upload(qb)
-    m, n = qa.rows, qb.rows
-    for dt in dtypes:
-        # the output row pitch must be a multiple of 16 bytes: pad it
-        per16 = 16 // torch.tensor([], dtype=dt).element_size()
-        ld = -(-n // per16) * per16
-        y = nv.gemm(A, B, out=torch.empty((m, ld), dtype=dt, device="cuda")[:, :n])
-        torch.cuda.synchronize()
-        gemm_check(y, ref, rn, cn, f"{what} {dt}")
+    m, n, k = qa.rows, qb.rows, qa.k
+    for use_ws in workspaces:
+        ws = None
+        if use_ws:
+            nbytes = nv.gemm_workspace_bytes(m, n, k)
+            if nbytes == 0:
+                continue
+            ws = torch.full((nbytes,), 0x7F, dtype=torch.uint8, device="cuda")  # garbage
+        for dt in dtypes:
+            # the output row pitch must be a multiple of 16 bytes: pad it
+            per16 = 16 // torch.tensor([], dtype=dt).element_size()
+            ld = -(-n // per16) * per16
+            y = nv.gemm(A, B, out=torch.empty((m, ld), dtype=dt, device="cuda")[:, :n],
+                        workspace=ws)
+            torch.cuda.synchronize()
+            gemm_check(y, ref, rn, cn, f"{what} {dt} workspace={use_ws}")
     assert nv.read_fault() == 0
 
 
@@ -96,3 +107,10 @@ def test_gemm_decode_shapes(nv, orc, m, k, n):
     from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
     cfg = wl.decode(m, k, n)
     run_case(nv, orc, cfg.x(), cfg.w(), dtypes=(torch.bfloat16,), what=cfg.name)
+
+
+@pytest.mark.parametrize("m", [1, 16, 17, 100, 255])
+def test_gemm_few_tokens_split_k(nv, orc, m):
+    """Few-token path with K split across CTAs (N = 1000: 8 weight tiles,
+    so most of the GPU works on K slices) and ragged token counts."""
+    run_case(nv, orc, gaussian(m, 2048, 7 * m), gaussian(1000, 2048, 11, 0.02), what=f"split m={m}")
