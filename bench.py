@@ -10,6 +10,9 @@ offline in a W4A4 checkpoint). Workloads:
   outlier    X 8192x5120 (8 channels x50) @ W 5120x5120        (default)
   gdn_fused  X 8192x5120 @ fused qkv|z|a|b 12384x5120 (fold done offline)
   mlp32k     X 32768x5120 -> gate_up 34816 -> silu*mul -> requant -> down 5120
+  mlp32k_fused  the same MLP with silu*mul + quantization of h fused into the
+             gate_up GEMM epilogue (h's static global calibrated offline)
+  decode:M:K:N  few-token GEMM, e.g. decode:1:5120:17408 (HBM-bound)
 Metric: TFLOP/s of the whole step (2*M*N*K per GEMM over quantize + GEMM
 time), with the GEMM's fraction of the dense FP4 tensor peak and the
 quantizer's GB/s alongside. Inputs stay resident in HBM; L2 (126 MB) is
@@ -172,15 +175,40 @@ def make_workload(name: str, rank: int):
                 "(per-module globals folded offline); quantize X + one fused GEMM")
         return dict(x=x, W=W, gemms=[(cfg.m, cfg.n, cfg.k)], desc=desc, kind="linear",
                     m=cfg.m, n=cfg.n, k=cfg.k)
-    if name == "mlp32k":
+    if name in ("mlp32k", "mlp32k_fused"):
         cfg = wl.mlp32k()
         x = cfg.x().cuda()
-        Wgu = nvfp4.quantize(cfg.w_gate_up().cuda())
         Wd = nvfp4.quantize(cfg.w_down().cuda())
-        desc = (f"mlp32k: X {cfg.m}x{cfg.d} -> gate_up {2 * cfg.ffn}x{cfg.d} -> silu*mul -> "
-                f"requant -> down {cfg.d}x{cfg.ffn}")
-        return dict(x=x, Wgu=Wgu, Wd=Wd, gemms=[(cfg.m, 2 * cfg.ffn, cfg.d), (cfg.m, cfg.d, cfg.ffn)],
-                    desc=desc, kind="mlp", m=cfg.m, n=cfg.d, k=cfg.d, ffn=cfg.ffn)
+        gemms = [(cfg.m, 2 * cfg.ffn, cfg.d), (cfg.m, cfg.d, cfg.ffn)]
+        if name == "mlp32k":
+            Wgu = nvfp4.quantize(cfg.w_gate_up().cuda())
+            desc = (f"mlp32k: X {cfg.m}x{cfg.d} -> gate_up {2 * cfg.ffn}x{cfg.d} -> silu*mul -> "
+                    f"requant (dynamic global) -> down {cfg.d}x{cfg.ffn}")
+            return dict(x=x, Wgu=Wgu, Wd=Wd, gemms=gemms, desc=desc, kind="mlp", m=cfg.m,
+                        n=cfg.d, k=cfg.d, ffn=cfg.ffn)
+        Wgi = nvfp4.quantize(nvfp4.interleave_gate_up(cfg.w_gate_up().cuda()))
+        # offline calibration of h's static global on this batch (unfused path)
+        A = nvfp4.quantize(x)
+        y = nvfp4.gemm(A, Wgi)
+        yb = y.view(cfg.m, cfg.ffn // 128, 2, 128)
+        h = nvfp4.silu_mul(torch.cat([yb[:, :, 0].reshape(cfg.m, cfg.ffn),
+                                      yb[:, :, 1].reshape(cfg.m, cfg.ffn)], 1).contiguous())
+        gh = nvfp4.Calibrator().observe(h).clone()
+        del y, yb, h, A
+        desc = (f"mlp32k_fused: X {cfg.m}x{cfg.d} -> gate_up {2 * cfg.ffn}x{cfg.d} with "
+                f"silu*mul + static-global NVFP4 quantization of h in the epilogue -> down "
+                f"{cfg.d}x{cfg.ffn}")
+        return dict(x=x, Wgi=Wgi, Wd=Wd, gh=gh, gemms=gemms, desc=desc, kind="mlp_fused",
+                    m=cfg.m, n=cfg.d, k=cfg.d, ffn=cfg.ffn)
+    if name.startswith("decode:"):
+        m, k, n = (int(v) for v in name.split(":")[1:])
+        cfg = wl.decode(m, k, n)
+        x = cfg.x().cuda()
+        W = nvfp4.quantize(cfg.w().cuda())
+        desc = (f"decode: X {m}x{k} -> quantize -> W4A4 GEMM vs W {n}x{k} NVFP4 "
+                "(few-token kernel, K split across the GPU)")
+        return dict(x=x, W=W, gemms=[(m, n, k)], desc=desc, kind="linear", m=m, n=n, k=k,
+                    decode=True)
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -196,15 +224,25 @@ class Step:
         m, k = wk["x"].shape
         self.A = nvfp4.NVFP4Tensor.empty(m, k, dev)
         self.ws = torch.empty(nvfp4.quantize_workspace_bytes(m, k), dtype=torch.uint8, device=dev)
+        self.gws = None
         if wk["kind"] == "linear":
             self.y = torch.empty((m, wk["W"].rows), dtype=torch.bfloat16, device=dev)
+            nb = nvfp4.gemm_workspace_bytes(m, wk["W"].rows, k)
+            if nb:
+                self.gws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        elif wk["kind"] == "mlp_fused":
+            ffn = wk["ffn"]
+            self.H = nvfp4.NVFP4Tensor.empty(m, ffn, dev)
+            self.y = torch.empty((m, wk["n"]), dtype=torch.bfloat16, device=dev)
         else:
             ffn = wk["ffn"]
             self.ygu = torch.empty((m, 2 * ffn), dtype=torch.bfloat16, device=dev)
             self.h = torch.empty((m, ffn), dtype=torch.bfloat16, device=dev)
             self.H = nvfp4.NVFP4Tensor.empty(m, ffn, dev)
             self.y = torch.empty((m, wk["n"]), dtype=torch.bfloat16, device=dev)
-        self.launches = 3 if wk["kind"] == "linear" else 9
+        self.launches = {"linear": 3, "mlp": 9, "mlp_fused": 4}[wk["kind"]]
+        if self.gws is not None:
+            self.launches += 2  # workspace clear + finalize of the K split
 
     def run(self, ev=None, x=None):
         nv, wk, s = self.nv, self.wk, self.s
@@ -214,8 +252,13 @@ class Step:
         nv.quantize(x, out=self.A, workspace=self.ws, stream=s)
         rec(1)
         if wk["kind"] == "linear":
-            nv.gemm(self.A, wk["W"], out=self.y, stream=s)
+            nv.gemm(self.A, wk["W"], out=self.y, workspace=self.gws, stream=s)
             rec(2)
+        elif wk["kind"] == "mlp_fused":
+            nv.gemm_swiglu_quant(self.A, wk["Wgi"], wk["gh"], out=self.H, stream=s)
+            rec(2)
+            nv.gemm(self.H, wk["Wd"], out=self.y, stream=s)
+            rec(3)
         else:
             nv.gemm(self.A, wk["Wgu"], out=self.ygu, stream=s)
             rec(2)
@@ -271,7 +314,7 @@ def run_gpu(args):
     step = Step(wk, stream)
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device="cuda")
     flops = sum(2 * m * n * k for (m, n, k) in wk["gemms"])
-    nph = 3 if wk["kind"] == "linear" else 5
+    nph = {"linear": 3, "mlp": 5, "mlp_fused": 4}[wk["kind"]]
 
     with torch.cuda.stream(stream):
         for _ in range(args.warmup):
@@ -348,6 +391,17 @@ def run_gpu(args):
 
     assert nvfp4.read_fault(stream) == 0
     traffic = dram_traffic(args.workload)
+    if wk.get("decode"):
+        mm, nn, kk = gemm0
+        gemm_bytes = nn * kk // 2 + nn * kk // 16 + mm * kk // 2 + mm * kk // 16 + mm * nn * 2
+        gemm_gbs = gemm_bytes / (gemm_avg_ms * 1e-3) / 1e9
+        roofline = {"bound": "hbm", "achieved": round(gemm_gbs, 1), "peak": pk["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(gemm_gbs / pk["hbm_gbs"], 4), "traffic": traffic,
+                    "kernel": "nvfp4::skinny::skinny_kernel",
+                    "peak_source": f"measured copy bandwidth ({pk['source']})",
+                    "algorithmic_bytes_per_launch": gemm_bytes}
+    else:
+        roofline = None
     out = {
         "metric": METRIC,
         "value": round(value, 2),
@@ -364,7 +418,7 @@ def run_gpu(args):
         "config": {"workload": wk["desc"], "gemms_mnk": wk["gemms"],
                    "l2": "flushed (256 MiB write) before every timed step, outside the events",
                    "parallelism": f"replicas x{world} (independent batches, no collective)"},
-        "roofline": {"bound": "tensor", "achieved": round(gemm_tflops, 1),
+        "roofline": roofline or {"bound": "tensor", "achieved": round(gemm_tflops, 1),
                      "peak": round(fp4_peak, 1), "unit": "TFLOP/s",
                      "frac": round(gemm_tflops / fp4_peak, 4),
                      "traffic": traffic,
@@ -389,7 +443,7 @@ def run_gpu(args):
         "clocks": clocks,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(args.workload, budget_s=args.cpu_seconds)
+        out["cpu_baseline"] = cpu_baseline(oracle_name(args.workload), budget_s=args.cpu_seconds)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist is not None:
@@ -431,6 +485,7 @@ def oracle_sample_step(orc, wk_cpu, rows):
     """One bounded sample of the step on the CPU oracle: quantize `rows` rows
     of X (dynamic global over the sample) and their FP64 GEMM rows."""
     import numpy as np
+    rows = min(rows, len(wk_cpu["x_bits"]))
     xs = wk_cpu["x_bits"][:rows]
     qa = orc.quantize(np.ascontiguousarray(xs))
     if wk_cpu["kind"] == "linear":
@@ -439,6 +494,15 @@ def oracle_sample_step(orc, wk_cpu, rows):
     yb = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     h = orc.silu_mul(yb)
     return orc.gemm(orc.quantize(h), wk_cpu["qd"])
+
+
+def oracle_name(workload: str) -> str:
+    """Workload whose oracle sample stands for this one (same arithmetic)."""
+    if workload.startswith("mlp32k"):
+        return "mlp32k"
+    if workload.startswith("decode:"):
+        return workload
+    return workload
 
 
 def oracle_workload(name):
@@ -458,6 +522,11 @@ def oracle_workload(name):
         mods = [orc.quantize(bits(w)) for w in cfg.weights()]
         return orc, dict(kind="linear", x_bits=bits(cfg.x()[:1024]), qw=orc.fuse_group(mods),
                          flops_per_row=2 * cfg.n * cfg.k)
+    if name.startswith("decode:"):
+        m, k, n = (int(v) for v in name.split(":")[1:])
+        cfg = wl.decode(m, k, n)
+        return orc, dict(kind="linear", x_bits=bits(cfg.x()), qw=orc.quantize(bits(cfg.w())),
+                         flops_per_row=2 * n * k)
     cfg = wl.mlp32k()
     return orc, dict(kind="mlp", x_bits=bits(cfg.x(rows=1024)),
                      qgu=orc.quantize(bits(cfg.w_gate_up())), qd=orc.quantize(bits(cfg.w_down())),
@@ -466,6 +535,7 @@ def oracle_workload(name):
 
 def cpu_baseline(name, budget_s=15.0, rows=128):
     orc, w = oracle_workload(name)
+    rows = min(rows, len(w["x_bits"]))
     oracle_sample_step(orc, w, 8)  # warm (builds/loads the oracle)
     t0 = time.perf_counter()
     reps = 0
@@ -486,8 +556,8 @@ def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    orc, w = oracle_workload(args.workload)
-    rows = args.ref_rows
+    orc, w = oracle_workload(oracle_name(args.workload))
+    rows = min(args.ref_rows, len(w["x_bits"]))
     for _ in range(args.warmup):
         oracle_sample_step(orc, w, 8)
     times = []
@@ -499,7 +569,9 @@ def run_reference(args):
     value = w["flops_per_row"] * rows / (ms * 1e-3) / 1e12
     wk_desc = {"outlier": "outlier: X 8192x5120 (8 channels x50) @ W 5120x5120",
                "gdn_fused": "gdn_fused: X 8192x5120 @ fused 12384x5120",
-               "mlp32k": "mlp32k: X 32768x5120 -> 34816 -> 17408 -> 5120"}[args.workload]
+               "mlp32k": "mlp32k: X 32768x5120 -> 34816 -> 17408 -> 5120",
+               "mlp32k_fused": "mlp32k (fused gate_up epilogue): X 32768x5120 -> 34816 -> "
+                               "17408 -> 5120"}.get(args.workload, args.workload)
     out = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -518,7 +590,8 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="outlier", choices=["outlier", "gdn_fused", "mlp32k"])
+    ap.add_argument("--workload", default="outlier",
+                    help="outlier | gdn_fused | mlp32k | mlp32k_fused | decode:M:K:N")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
