@@ -160,9 +160,11 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k,
                                     size_t workspace_bytes,
                                     nvfp4_stream_t stream);
 
-/* Workspace bytes nvfp4_gemm can use: m*n*4 for m <= 64 (few-token GEMMs
- * split K across CTAs and sum FP32 partials there), else 0. Passing less (or
- * NULL) is allowed and only disables the split. */
+/* Workspace bytes nvfp4_gemm can use: for m <= 64, 16*ceil(n/128) bytes of
+ * split counters (rounded up to 256) plus 8*m*n*4 bytes for up to 8 FP32
+ * slabs of Y (few-token GEMMs split K across CTAs and add the slabs in a fixed
+ * order); else 0. Passing less (or NULL) is allowed and only disables the
+ * split. */
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -181,9 +183,13 @@ size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *            16 bytes) and k >= 32.
  *   a_codes, b_codes: 16-byte aligned. a_sf, b_sf: 16-byte aligned.
  *   workspace  device scratch, nvfp4_gemm_workspace_bytes(m,n,k) bytes,
- *              16-byte aligned, or NULL; contents need no initialisation.
+ *              16-byte aligned, or NULL; contents need no initialisation
+ *              (the call zeroes the split counters itself).
  * m <= 64 runs the few-token kernel (weights on the MMA's 128-row side,
- * tokens as its N); larger m the paired-CTA 256x256-tile kernel.
+ * tokens as its N); larger m the paired-CTA 256x256-tile kernel. Results do
+ * not depend on the run: split-K slices are summed in slice order.
+ * The kernel is launched with programmatic stream serialisation; it reads and
+ * writes global memory only after the previous kernel in the stream finished.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
  */
 nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
@@ -192,6 +198,40 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
                         int y_dtype, int64_t ldy, int64_t m, int64_t n,
                         int64_t k, void* workspace, size_t workspace_bytes,
                         nvfp4_stream_t stream);
+
+/* Workspace bytes of nvfp4_linear: the quantized activations (codes, scales,
+ * global), the amax pass's partial maxima and, for m <= 64, the few-token
+ * GEMM's split counters and slabs. 0 for invalid sizes. */
+size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
+
+/*
+ * nvfp4_linear — the W4A4 linear layer in one call (news §02: activations are
+ * quantized to NVFP4 on the fly and multiplied with NVFP4 weights on the
+ * 4-bit tensor cores): Y = dequant(quantize(X)) @ dequant(W)^T, i.e.
+ * nvfp4_quantize of X into the workspace followed by nvfp4_gemm, with
+ * identical results. The GEMM is launched to start while the quantizer runs:
+ * its set-up and its first weight tiles overlap the quantization. This
+ * relies on W, w_sf and w_global being written before the call (by work
+ * already in the stream or earlier), never by a kernel launched in between.
+ *   x         device bf16 [m][ldx], 16-byte aligned, ldx >= k, ldx % 8 == 0.
+ *   x_global  NULL: dynamic global scale of X (amax pass); else a device FP32
+ *             static global (e.g. from nvfp4_calibrate_global).
+ *   w_codes, w_sf, w_global  weights [n][k] in NVFP4 (as nvfp4_gemm's B).
+ *   y, y_dtype, ldy          as nvfp4_gemm.
+ *   m, n >= 1; k % 32 == 0.
+ *   workspace  device scratch of nvfp4_linear_workspace_bytes(m,n,k) bytes,
+ *              256-byte aligned, owned by the caller, not shared with a call
+ *              that may run at the same time, and zero-filled before its
+ *              first use: each call leaves the bytes that must start at zero
+ *              zeroed again (after a kernel timeout, zero it again).
+ * Errors: INVALID_ARG (null pointer, bad size, short workspace), MISALIGNED,
+ * UNSUPPORTED (k % 32 != 0, sizes >= 2^31), CUDA.
+ */
+nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
+                          const float* x_global, const uint8_t* w_codes,
+                          const uint8_t* w_sf, const float* w_global, int64_t n,
+                          void* y, int y_dtype, int64_t ldy, void* workspace,
+                          size_t workspace_bytes, nvfp4_stream_t stream);
 
 /*
  * nvfp4_gemm_swiglu_quant — gate_up projection of a W4A4 gated MLP with the

@@ -10,8 +10,17 @@
 //
 // One CTA per SM, persistent over work units (128 weight rows x one slice of
 // K). When the weight tiles alone cannot occupy the GPU, K is split across
-// CTAs and each slice adds its FP32 partial into a zeroed workspace with
-// red.global.add; a finalize kernel converts the sum.
+// CTAs (at most kMaxSplits slices): each slice writes its FP32 partial
+// (already scaled by 1/(g_a g_b)) to its own workspace slab; then each
+// epilogue warp counts itself in on the counter of its 32 output columns,
+// and the warp that arrives last for those columns sums the slabs in slice
+// order, writes Y and resets the counter. The result is the same on every
+// run, and no warp ever waits for another.
+// Launched with programmatic stream serialisation: tensor-memory allocation
+// and barrier set-up overlap the previous kernel; every global access waits
+// for it, except that, when the caller guarantees the weights were written
+// before that kernel started (`early_w`), the first ring's worth of weight
+// tiles is requested before the wait.
 //   warp 0     TMA producer: W tile (128 rows x 128 B, 128-byte swizzle), the
 //              token tile (BNT rows), and both tiles' scale atoms, into a
 //              ring of up to 8 stages.
@@ -51,6 +60,8 @@ constexpr uint32_t SF_BUF_COLS = 48;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 constexpr size_t kSmemBudget = 220 * 1024;
+constexpr int kMaxSplits = 8;     // K slices per weight tile
+constexpr int kSumTokens = 16;    // tokens summed per round of slab loads
 
 enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, kFaultScales = 128u };
 
@@ -82,7 +93,9 @@ struct Params {
   void* y;                  // direct mode: [M][ldy] bf16 / fp32
   int64_t ldy;
   int y_fp32;
-  float* partial;           // split mode: [M][N] FP32, zeroed before launch
+  float* partial;           // split mode: [splits][M][N] FP32 slabs
+  unsigned int* tile_count; // split mode: [num_w_tiles * 4], zero before and after a launch
+  int early_w;              // weights may be read before the previous kernel finishes
 };
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
@@ -118,9 +131,21 @@ __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[3
       : "memory");
 }
 
-__device__ __forceinline__ void red_add_f32(float* p, float v) {
-  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(v) : "memory");
-}
+// Issue order of the producer: (unit, k-tile) pairs of this CTA.
+struct WorkIter {
+  int u, kt, k1, wt;
+  __device__ __forceinline__ void start(int unit, const Params& p, int num_units) {
+    u = unit;
+    if (u < num_units) {
+      wt = u % p.num_w_tiles;
+      kt = (u / p.num_w_tiles) * p.k_tiles_per_split;
+      k1 = min(p.num_k_tiles, kt + p.k_tiles_per_split);
+    }
+  }
+  __device__ __forceinline__ void next(const Params& p, int num_units) {
+    if (++kt >= k1) start(u + static_cast<int>(gridDim.x), p, num_units);
+  }
+};
 
 template <int BNT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
@@ -179,29 +204,49 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0;
       bool aborted = false;
-      for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-        const int wt = u % p.num_w_tiles, sp = u / p.num_w_tiles;
-        const int k0 = sp * p.k_tiles_per_split;
-        const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
-        for (int kt = k0; kt < k1; ++kt) {
-          if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer)) {
-            aborted = true;
-            break;
-          }
-          pending &= ~(1u << stage);
-          uint8_t* st = smem + stage * C::STAGE_BYTES;
-          ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
-          ptx::tma_load_2d(st, &tmW, &full[stage], kt * BK_BYTES, wt * BW);
-          ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], kt * BK_BYTES, 0);
-          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, kt * 4, wt);
-          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
-                           kt * 4, 0);
-          pending |= 1u << stage;
-          pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+      WorkIter it;
+      it.start(blockIdx.x, p, num_units);
+      // The first ring's worth of stages needs no empty-slot wait. With
+      // early_w their weight halves are requested before the grid-dependency
+      // wait, the token halves after it.
+      int npre = 0;
+      if (p.early_w) {
+        WorkIter w = it;
+        for (; npre < C::STAGES && w.u < num_units; ++npre, w.next(p, num_units)) {
+          uint8_t* st = smem + npre * C::STAGE_BYTES;
+          ptx::mbar_arrive_expect_tx(&full[npre], C::STAGE_RAW);
+          ptx::tma_load_2d(st, &tmW, &full[npre], w.kt * BK_BYTES, w.wt * BW);
+          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4, w.wt);
+        }
+      }
+      ptx::grid_dep_wait();
+      for (int i = 0; i < npre; ++i, it.next(p, num_units)) {
+        uint8_t* st = smem + i * C::STAGE_BYTES;
+        ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[i], it.kt * BK_BYTES, 0);
+        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[i], 0,
+                         it.kt * 4, 0);
+        pending |= 1u << i;
+      }
+      stage = static_cast<uint32_t>(npre % C::STAGES);
+      phase = static_cast<uint32_t>(npre / C::STAGES);
+      for (; it.u < num_units; it.next(p, num_units)) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer)) {
+          aborted = true;
+          break;
+        }
+        pending &= ~(1u << stage);
+        uint8_t* st = smem + stage * C::STAGE_BYTES;
+        ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
+        ptx::tma_load_2d(st, &tmW, &full[stage], it.kt * BK_BYTES, it.wt * BW);
+        ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], it.kt * BK_BYTES, 0);
+        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, it.kt * 4, it.wt);
+        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
+                         it.kt * 4, 0);
+        pending |= 1u << stage;
+        pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == C::STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
       if (aborted)
@@ -312,16 +357,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue --
+    ptx::grid_dep_wait();  // the globals come from earlier kernels; Y may be in use
     const int q = warp & 3;  // tensor-memory lane quarter (warps 4..7 -> 0..3)
     const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
     uint32_t acc_phase = 0;
     for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
       const int wt = u % p.num_w_tiles;
+      const int sp = u / p.num_w_tiles;
       if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue)) break;
       ptx::tc_fence_after();
       const int n = wt * BW + q * 32 + lane;   // this thread's output column
       const bool n_ok = n < p.N;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      float* slab = p.splits > 1 ? p.partial + static_cast<int64_t>(sp) * p.M * p.N : nullptr;
 #pragma unroll
       for (int c0 = 0; c0 < BNT; c0 += 32) {
         uint32_t r[32];
@@ -337,8 +385,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int m = c0 + i;                 // token
           if (m >= p.M || !n_ok) continue;
           const float v = __uint_as_float(r[i]) * alpha;
-          if (p.partial != nullptr) {
-            red_add_f32(p.partial + static_cast<int64_t>(m) * p.N + n, v);
+          if (p.splits > 1) {
+            slab[static_cast<int64_t>(m) * p.N + n] = v;
           } else if (p.y_fp32) {
             reinterpret_cast<float*>(p.y)[static_cast<int64_t>(m) * p.ldy + n] = v;
           } else {
@@ -351,6 +399,45 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tmem_empty);
       acc_phase ^= 1u;
+      if (p.splits > 1) {
+        // count this slice in for these 32 columns; the last one sums them
+        __threadfence();
+        __syncwarp();
+        uint32_t last = 0;
+        if (lane == 0)
+          last = atomicAdd(p.tile_count + wt * 4 + q, 1u) == static_cast<unsigned>(p.splits - 1);
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (last) {
+          __threadfence();
+          if (n_ok) {
+            for (int m0 = 0; m0 < p.M; m0 += kSumTokens) {
+              float v[kSumTokens][kMaxSplits];
+#pragma unroll
+              for (int i = 0; i < kSumTokens; ++i)
+#pragma unroll
+                for (int s2 = 0; s2 < kMaxSplits; ++s2)
+                  v[i][s2] = (s2 < p.splits && m0 + i < p.M)
+                                 ? __ldcg(p.partial + (static_cast<int64_t>(s2) * p.M + m0 + i) *
+                                                          p.N + n)
+                                 : 0.0f;
+#pragma unroll
+              for (int i = 0; i < kSumTokens; ++i) {
+                if (m0 + i >= p.M) break;
+                float acc = v[i][0];
+#pragma unroll
+                for (int s2 = 1; s2 < kMaxSplits; ++s2)
+                  if (s2 < p.splits) acc += v[i][s2];
+                const int64_t o = static_cast<int64_t>(m0 + i) * p.ldy + n;
+                if (p.y_fp32)
+                  reinterpret_cast<float*>(p.y)[o] = acc;
+                else
+                  reinterpret_cast<__nv_bfloat16*>(p.y)[o] = __float2bfloat16_rn(acc);
+              }
+            }
+          }
+          if (lane == 0) p.tile_count[wt * 4 + q] = 0u;  // ready for the next call
+        }
+      }
     }
   }
 
@@ -360,22 +447,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
-  }
-}
-
-// Split mode: Y = the FP32 sums (already scaled by 1/(g_a g_b)), converted.
-__global__ void __launch_bounds__(256)
-    finalize_kernel(const float* __restrict__ partial, int64_t m, int64_t n, void* y,
-                    int64_t ldy, int y_fp32) {
-  const int64_t total = m * n;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = i / n, c = i - r * n;
-    const float v = partial[i];
-    if (y_fp32)
-      reinterpret_cast<float*>(y)[r * ldy + c] = v;
-    else
-      reinterpret_cast<__nv_bfloat16*>(y)[r * ldy + c] = __float2bfloat16_rn(v);
   }
 }
 

@@ -45,6 +45,11 @@
 // SwiGLU expression, h rounded to bf16) and quantizes h to NVFP4 with a
 // calibrated static global using the quantizer's arithmetic, writing codes
 // and swizzled scales of h instead of the 2*ffn-wide bf16 output.
+// Launched with programmatic stream serialisation: barrier set-up and
+// tensor-memory allocation overlap the previous kernel in the stream; the
+// producer and the epilogue wait for it before touching global memory, except
+// that with `early_w` (weights known to be written before that kernel began)
+// the first ring's worth of B tiles and scales is requested before the wait.
 // Every mbarrier wait is bounded in time; on expiry the kernel records a fault
 // word, both CTAs of the pair stop, in-flight copies and MMAs are drained
 // (again with a bound) and tensor memory is released before the CTAs exit.
@@ -116,6 +121,7 @@ struct Params {
   uint8_t* h_sf;           // swizzled scales of [M][ffn]
   int64_t h_atoms;         // 512-byte atoms per 128-row block = ffn / 64
   int m_pad;               // rows of the scale buffer = ceil(M/128)*128
+  int early_w;             // B may be read before the previous kernel finishes
 };
 
 // Band rasterization: consecutive tiles walk GROUP_M M-tiles down one N band,
@@ -330,32 +336,67 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0;
       uint32_t pending = 0, pending_parity = 0;  // stages loaded, not yet seen free
       bool aborted = false;
-      for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
-        int mb, nb;
-        tile_coords(t, p, mb, nb);
-        const int arow = mb * BM + static_cast<int>(rank) * HALF;
-        const int brow = nb * BN + static_cast<int>(rank) * HALF;
-        for (int kt = 0; kt < p.num_k_tiles; ++kt) {
-          if (!wait_bounded(&empty[stage], phase ^ 1u, ab, kFaultProducer)) {
-            aborted = true;
-            break;
-          }
-          pending &= ~(1u << stage);
-          uint8_t* st = smem + stage * STAGE_BYTES;
-          // the even CTA's barrier counts both CTAs' bytes of this stage
-          const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(&full[stage]), 0);
-          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-          ptx::tma_load_2d_pair(st, &tmA, bar, kt * BK_BYTES, arow);
-          ptx::tma_load_2d_pair(st + A_BYTES, &tmB, bar, kt * BK_BYTES, brow);
-          ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES, &tmSFA, bar, 0, kt * 4,
-                                mb * 2 + static_cast<int>(rank));
-          ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tmSFB, bar, 0, kt * 4, nb * 2);
-          pending |= 1u << stage;
-          pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1u;
-          }
+      // issue order: (tile, k-tile) pairs of this CTA pair
+      struct Item {
+        int t, kt, mb, nb;
+      };
+      auto first = [&](int t) {
+        Item it{t, 0, 0, 0};
+        if (t < num_tiles) tile_coords(t, p, it.mb, it.nb);
+        return it;
+      };
+      auto next = [&](Item it) {
+        if (++it.kt == p.num_k_tiles) it = first(it.t + num_pairs);
+        return it;
+      };
+      // the even CTA's barrier counts both CTAs' bytes of a stage
+      auto load_b = [&](const Item& it, uint32_t s) {
+        uint8_t* st = smem + s * STAGE_BYTES;
+        const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
+        ptx::tma_load_2d_pair(st + A_BYTES, &tmB, bar, it.kt * BK_BYTES,
+                              it.nb * BN + static_cast<int>(rank) * HALF);
+        ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tmSFB, bar, 0, it.kt * 4,
+                              it.nb * 2);
+      };
+      auto load_a = [&](const Item& it, uint32_t s) {
+        uint8_t* st = smem + s * STAGE_BYTES;
+        const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
+        ptx::tma_load_2d_pair(st, &tmA, bar, it.kt * BK_BYTES,
+                              it.mb * BM + static_cast<int>(rank) * HALF);
+        ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES, &tmSFA, bar, 0, it.kt * 4,
+                              it.mb * 2 + static_cast<int>(rank));
+      };
+      Item it = first(pair);
+      // The ring's first pass needs no empty-slot wait; with early_w its B
+      // halves are requested before the grid-dependency wait.
+      int npre = 0;
+      if (p.early_w) {
+        for (Item w = it; npre < STAGES && w.t < num_tiles; ++npre, w = next(w)) {
+          if (leader) ptx::mbar_arrive_expect_tx(&full[npre], 2 * STAGE_BYTES);
+          load_b(w, static_cast<uint32_t>(npre));
+        }
+      }
+      ptx::grid_dep_wait();
+      for (int i = 0; i < npre; ++i, it = next(it)) {
+        load_a(it, static_cast<uint32_t>(i));
+        pending |= 1u << i;
+      }
+      stage = static_cast<uint32_t>(npre % STAGES);
+      phase = static_cast<uint32_t>(npre / STAGES);
+      for (; it.t < num_tiles; it = next(it)) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, ab, kFaultProducer)) {
+          aborted = true;
+          break;
+        }
+        pending &= ~(1u << stage);
+        if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+        load_a(it, stage);
+        load_b(it, stage);
+        pending |= 1u << stage;
+        pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
         }
       }
       if (aborted && leader) {
@@ -451,6 +492,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // -------------------------------------------------------------- epilogue --
+    ptx::grid_dep_wait();  // globals from earlier kernels; Y / h may still be in use
     float* rtab = reinterpret_cast<float*>(smem + RTAB_OFF);
     if (p.fused) {
       // E4M3 code -> g_h / dec(code), as the quantizer tabulates it

@@ -4,6 +4,10 @@
 // on the host (returning a status before anything is launched), builds the
 // TMA descriptors of the GEMM and launches on the caller's stream. Nothing is
 // allocated and no call synchronises with the host except nvfp4_read_fault.
+// The quantizer's second kernel and the GEMMs are launched with programmatic
+// stream serialisation (each kernel waits on the device for its predecessor
+// before touching global memory), so a launch and its set-up overlap the
+// previous kernel's tail.
 #include "nvfp4.h"
 
 #include <cuda.h>
@@ -13,6 +17,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include "fold.cuh"
 #include "gemm_sm100.cuh"
@@ -80,6 +85,53 @@ nvfp4_status launch_status() {
 
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+// Launch with programmatic stream serialisation (and a cluster shape when
+// cluster_x > 1). The kernel must call grid_dep_wait() before any access to
+// global memory that earlier work in the stream produces or consumes.
+template <typename... KArgs, typename... Args>
+nvfp4_status launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t smem,
+                        cudaStream_t s, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  std::memset(&cfg, 0, sizeof cfg);
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  std::memset(attr, 0, sizeof attr);
+  unsigned na = 0;
+  attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[na].val.programmaticStreamSerializationAllowed = 1;
+  ++na;
+  if (cluster_x > 1) {
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = cluster_x;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = na;
+  if (cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) != cudaSuccess) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+// Few-token GEMM workspace: split counters (4 per 128 weight rows), then up
+// to kMaxSplits FP32 slabs of Y.
+size_t skinny_counter_bytes(int64_t n) {
+  return round_up(static_cast<size_t>(ceil_div(n, 128)) * 4 * sizeof(unsigned int), 256);
+}
+size_t skinny_workspace_bytes(int64_t m, int64_t n) {
+  return skinny_counter_bytes(n) + static_cast<size_t>(nvfp4::skinny::kMaxSplits) *
+                                       static_cast<size_t>(m) * static_cast<size_t>(n) *
+                                       sizeof(float);
+}
+
 // CTAs of the amax pass: enough that every thread streams ~8 16-byte chunks
 // (the contiguous path is flat over elements, the strided one a warp per
 // row), at most 2 per SM. Sizing by rows alone starved few-row inputs.
@@ -113,6 +165,42 @@ nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
   }
   *out = st->noalloc_partials;
   return NVFP4_OK;
+}
+
+// Dynamic or static NVFP4 quantization of x (arguments already checked):
+// the amax pass (dynamic only) into `partials` (at most max_parts CTAs),
+// then the quantizer, launched to overlap the amax pass's tail.
+nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx,
+                             const float* global_in, uint8_t* codes, uint8_t* sf,
+                             float* global_out, float* partials, int64_t max_parts,
+                             const DeviceState* st, cudaStream_t s) {
+  using namespace nvfp4::quant;
+  int nparts = 0;
+  if (global_in == nullptr) {
+    const int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
+    if (blocks > max_parts) return NVFP4_ERR_UNSUPPORTED;
+    nparts = static_cast<int>(blocks);
+    amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
+                                                partials);
+    if (nvfp4_status e = launch_status()) return e;
+  }
+  QuantArgs a;
+  a.x = static_cast<const uint16_t*>(x);
+  a.rows = rows;
+  a.k = k;
+  a.ldx = ldx;
+  a.global_in = global_in;
+  a.partials = partials;
+  a.nparts = nparts;
+  a.codes = codes;
+  a.sf = sf;
+  a.global_out = global_out;
+  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
+  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
+  const int64_t cap = static_cast<int64_t>(st->sms) * kQuantBlocksPerSM;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(quantize_kernel, static_cast<unsigned>(blocks), kQuantThreads, 0, s, 1u, a);
 }
 
 }  // namespace
@@ -163,36 +251,9 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
   int dev;
   DeviceState* st;
   if (nvfp4_status e = current_device(&dev, &st)) return e;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
-  int nparts = 0;
-  if (dynamic) {
-    int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
-    if (blocks > kMaxPartials) blocks = kMaxPartials;
-    if (blocks < 1) blocks = 1;
-    nparts = static_cast<int>(blocks);
-    amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
-                                                static_cast<float*>(workspace));
-    if (nvfp4_status e = launch_status()) return e;
-  }
-  QuantArgs a;
-  a.x = static_cast<const uint16_t*>(x);
-  a.rows = rows;
-  a.k = k;
-  a.ldx = ldx;
-  a.global_in = global_in;
-  a.partials = static_cast<const float*>(workspace);
-  a.nparts = nparts;
-  a.codes = codes;
-  a.sf = sf;
-  a.global_out = global_out;
-  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
-  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
-  const int64_t cap = static_cast<int64_t>(st->sms) * kQuantBlocksPerSM;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  quantize_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(a);
-  return launch_status();
+  return quantize_launch(x, rows, k, ldx, global_in, codes, sf, global_out,
+                         static_cast<float*>(workspace), kMaxPartials, st,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k, int64_t ldx,
@@ -211,35 +272,8 @@ nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t rows, int64_t k, int6
   if (nvfp4_status e = current_device(&dev, &st)) return e;
   float* partials = nullptr;
   if (nvfp4_status e = noalloc_scratch(st, &partials)) return e;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-
-  int nparts = 0;
-  if (global_in == nullptr) {
-    const int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
-    if (blocks > NVFP4_NOALLOC_MAX_PARTIALS) return NVFP4_ERR_UNSUPPORTED;
-    nparts = static_cast<int>(blocks);
-    amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
-                                                partials);
-    if (nvfp4_status e = launch_status()) return e;
-  }
-  QuantArgs a;
-  a.x = static_cast<const uint16_t*>(x);
-  a.rows = rows;
-  a.k = k;
-  a.ldx = ldx;
-  a.global_in = global_in;
-  a.partials = partials;
-  a.nparts = nparts;
-  a.codes = codes;
-  a.sf = sf;
-  a.global_out = global_out;
-  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
-  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
-  const int64_t cap = static_cast<int64_t>(st->sms) * kQuantBlocksPerSM;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  quantize_kernel<<<static_cast<unsigned>(blocks), kQuantThreads, 0, s>>>(a);
-  return launch_status();
+  return quantize_launch(x, rows, k, ldx, global_in, codes, sf, global_out, partials,
+                         NVFP4_NOALLOC_MAX_PARTIALS, st, reinterpret_cast<cudaStream_t>(stream));
 }
 
 nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k, int64_t ldx,
@@ -272,8 +306,8 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k, int6
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   (void)k;
   if (m < 1 || n < 1) return 0;
-  // few-token GEMMs split K across CTAs and sum FP32 partials of Y here
-  return m <= 64 ? static_cast<size_t>(m) * static_cast<size_t>(n) * sizeof(float) : 0;
+  // few-token GEMMs split K across CTAs: split counters and FP32 slabs of Y
+  return m <= 64 ? skinny_workspace_bytes(m, n) : 0;
 }
 
 }  // extern "C"
@@ -340,19 +374,24 @@ nvfp4_status launch_skinny(DeviceState* st, int bit, const CUtensorMap& tmW, con
       st->skinny_smem_set |= 1u << bit;
     }
   }
-  nvfp4::skinny::skinny_kernel<BNT><<<grid, nvfp4::skinny::NUM_THREADS, Cfg<BNT>::SMEM_BYTES, s>>>(
-      tmW, tmX, tmSFW, tmSFX, p);
-  return launch_status();
+  return launch_pdl(nvfp4::skinny::skinny_kernel<BNT>, static_cast<unsigned>(grid),
+                    nvfp4::skinny::NUM_THREADS, Cfg<BNT>::SMEM_BYTES, s, 1u, tmW, tmX, tmSFW,
+                    tmSFX, p);
 }
 
 // Few tokens (m <= 64): Y^T = B A^T with the weights on the MMA's 128-row
 // side and the tokens as its N; K split across CTAs when the weight tiles
-// cannot fill the GPU and a workspace for the FP32 partial sums is given.
+// cannot fill the GPU and a workspace (skinny_workspace_bytes) is given.
+// The split counters at the workspace's start are zeroed here when
+// `zero_counters`, else the caller guarantees they are zero (every call
+// leaves them so). `early_w`: the weights were written before the previous
+// kernel in the stream started, so the kernel may read them before it ends.
 nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                          const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
                          void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
-                         void* workspace, size_t workspace_bytes, cudaStream_t s) {
+                         void* workspace, size_t workspace_bytes, bool zero_counters,
+                         int early_w, cudaStream_t s) {
   using namespace nvfp4::skinny;
   const int bnt = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
   CUtensorMap tmW, tmX, tmSFW, tmSFX;
@@ -376,19 +415,24 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   p.ldy = ldy;
   p.y_fp32 = y_dtype;
   p.partial = nullptr;
+  p.tile_count = nullptr;
+  p.early_w = early_w;
   int splits = 1;
-  const size_t need = static_cast<size_t>(m) * static_cast<size_t>(n) * sizeof(float);
-  if (workspace != nullptr && workspace_bytes >= need && aligned(workspace, 16)) {
+  if (workspace != nullptr && workspace_bytes >= skinny_workspace_bytes(m, n) &&
+      aligned(workspace, 16)) {
     splits = st->sms / p.num_w_tiles;
     if (splits > p.num_k_tiles) splits = p.num_k_tiles;
+    if (splits > kMaxSplits) splits = kMaxSplits;
     if (splits < 1) splits = 1;
   }
   p.k_tiles_per_split = static_cast<int>(ceil_div(p.num_k_tiles, splits));
   splits = static_cast<int>(ceil_div(p.num_k_tiles, p.k_tiles_per_split));  // no empty slice
   p.splits = splits;
   if (splits > 1) {
-    p.partial = static_cast<float*>(workspace);
-    if (cudaMemsetAsync(workspace, 0, need, s) != cudaSuccess) {
+    p.tile_count = static_cast<unsigned int*>(workspace);
+    p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                         skinny_counter_bytes(n));
+    if (zero_counters && cudaMemsetAsync(workspace, 0, skinny_counter_bytes(n), s) != cudaSuccess) {
       cudaGetLastError();
       return NVFP4_ERR_CUDA;
     }
@@ -403,12 +447,7 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
     case 128: e = launch_skinny<128>(st, 3, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
     default: e = launch_skinny<256>(st, 4, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
   }
-  if (e != NVFP4_OK || splits == 1) return e;
-  int64_t blocks = ceil_div(m * n, 256);
-  if (blocks > static_cast<int64_t>(st->sms) * 8) blocks = static_cast<int64_t>(st->sms) * 8;
-  finalize_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(
-      static_cast<const float*>(workspace), m, n, y, ldy, y_dtype);
-  return launch_status();
+  return e;
 }
 
 // The paired-CTA kernel (cta_group::2, 256x256 tiles): M, N, K, tile counts
@@ -452,24 +491,8 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   // one CTA pair (cluster of 2 SMs) per 256x256 tile at a time, persistent
   const int64_t max_pairs = st->sms / 2;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
-  cudaLaunchConfig_t cfg;
-  std::memset(&cfg, 0, sizeof cfg);
-  cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs), 1, 1);
-  cfg.blockDim = dim3(NUM_THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 2;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, gemm_kernel, tmA, tmB, tmSFA, tmSFB, tmY, p) != cudaSuccess) {
-    cudaGetLastError();
-    return NVFP4_ERR_CUDA;
-  }
-  return launch_status();
+  return launch_pdl(gemm_kernel, static_cast<unsigned>(2 * pairs), NUM_THREADS, SMEM_BYTES,
+                    stream, 2u, tmA, tmB, tmSFA, tmSFB, tmY, p);
 }
 
 }  // namespace
@@ -499,7 +522,8 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   if (nvfp4_status e = get_encoder(&enc)) return e;
   if (m <= 64)
     return gemm_skinny(enc, st, a_codes, a_sf, a_global, b_codes, b_sf, b_global, y, y_dtype, ldy,
-                       m, n, k, workspace, workspace_bytes, reinterpret_cast<cudaStream_t>(stream));
+                       m, n, k, workspace, workspace_bytes, true, 0,
+                       reinterpret_cast<cudaStream_t>(stream));
 
   nvfp4::gemm::Params p;
   std::memset(&p, 0, sizeof p);
@@ -510,6 +534,62 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   p.y_fp32 = y_dtype;
   return gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, n, k, p,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
+  if (m < 1 || n < 1 || k < 32 || k % 32 != 0) return 0;
+  size_t b = m <= 64 ? round_up(skinny_workspace_bytes(m, n), 256) : 0;
+  b += round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);  // codes
+  b += round_up(nvfp4_sf_bytes(m, k), 256);                                // scales
+  b += 256;                                                                // global
+  b += static_cast<size_t>(nvfp4::quant::kMaxPartials) * sizeof(float);     // amax partials
+  return b;
+}
+
+nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
+                          const float* x_global, const uint8_t* w_codes, const uint8_t* w_sf,
+                          const float* w_global, int64_t n, void* y, int y_dtype, int64_t ldy,
+                          void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (!x || !w_codes || !w_sf || !w_global || !y || !workspace) return NVFP4_ERR_INVALID_ARG;
+  if (m < 1 || n < 1 || k < 1 || (y_dtype != 0 && y_dtype != 1) || ldy < n || ldx < k)
+    return NVFP4_ERR_INVALID_ARG;
+  if (k % 32 != 0 || m >= (int64_t{1} << 31) || n >= (int64_t{1} << 31) ||
+      k >= (int64_t{1} << 31))
+    return NVFP4_ERR_UNSUPPORTED;
+  const int64_t esize = y_dtype == 0 ? 2 : 4;
+  if (ldx % 8 != 0 || !aligned(x, 16) || !aligned(w_codes, 16) || !aligned(w_sf, 16) ||
+      !aligned(y, 16) || (ldy * esize) % 16 != 0 || !aligned(w_global, 4) ||
+      !aligned(x_global, 4) || !aligned(workspace, 256))
+    return NVFP4_ERR_MISALIGNED;
+  if (workspace_bytes < nvfp4_linear_workspace_bytes(m, n, k)) return NVFP4_ERR_INVALID_ARG;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (nvfp4_status e = get_encoder(&enc)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // workspace: [split counters + slabs (m <= 64)][codes][scales][global][partials]
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  const size_t split_bytes = m <= 64 ? round_up(skinny_workspace_bytes(m, n), 256) : 0;
+  uint8_t* a_codes = w + split_bytes;
+  uint8_t* a_sf = a_codes + round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);
+  float* a_global = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(m, k), 256));
+  float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a_global) + 256);
+  if (nvfp4_status e = quantize_launch(x, m, k, ldx, x_global, a_codes, a_sf, a_global, partials,
+                                       nvfp4::quant::kMaxPartials, st, s))
+    return e;
+  if (m <= 64)
+    return gemm_skinny(enc, st, a_codes, a_sf, a_global, w_codes, w_sf, w_global, y, y_dtype, ldy,
+                       m, n, k, w, skinny_workspace_bytes(m, n), false, 1, s);
+  nvfp4::gemm::Params p;
+  std::memset(&p, 0, sizeof p);
+  p.a_global = a_global;
+  p.b_global = w_global;
+  p.y = y;
+  p.ldy = ldy;
+  p.y_fp32 = y_dtype;
+  p.early_w = 1;
+  return gemm_paired(enc, st, a_codes, a_sf, w_codes, w_sf, m, n, k, p, s);
 }
 
 nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf,

@@ -6,6 +6,9 @@
 // Convention (FP32, round-to-nearest-even at every step):
 //   g = 2688 / amax;  s = E4M3(amax_b / 6 * g);  code = E2M1(x * (g / dec(s))).
 //
+// Both kernels wait for the previous kernel in the stream before touching
+// global memory, so they may be launched with programmatic stream
+// serialisation (the next kernel's launch then overlaps this one's tail).
 // Two kernels:
 //   amax_kernel      one pass over x, one partial max per CTA (no atomics, so
 //                    the workspace needs no initialisation);
@@ -64,6 +67,8 @@ __device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
 __global__ void __launch_bounds__(kAmaxThreads)
     amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ldx,
                 float* __restrict__ partials) {
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -122,6 +127,8 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs a) {
+  ptx::grid_dep_wait();    // partials / static global / x come from earlier kernels
+  ptx::grid_dep_launch();
   __shared__ float s_g;
   __shared__ float s_rtab[128];
   __shared__ uint32_t s_red[kQuantThreads / 32];
@@ -226,6 +233,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
 __global__ void __launch_bounds__(256)
     calibrate_kernel(const float* __restrict__ partials, int nparts, float* running_amax,
                      float* global_out) {
+  ptx::grid_dep_wait();
+  ptx::grid_dep_launch();
   __shared__ uint32_t s_red[8];
   uint32_t m = 0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, __float_as_uint(partials[i]));

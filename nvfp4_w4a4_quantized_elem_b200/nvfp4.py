@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPO
 # every symbol include/nvfp4.h declares
 EXPORTS = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_quantize_workspace_bytes",
            "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_calibrate_global",
-           "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_gemm_swiglu_quant",
+           "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_linear_workspace_bytes",
+           "nvfp4_linear", "nvfp4_gemm_swiglu_quant",
            "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault")
 
 _lib = None
@@ -60,6 +61,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_calibrate_global": (I, [P, I64, I64, I64, P, P, P, SZ, P]),
             "nvfp4_gemm_workspace_bytes": (SZ, [I64, I64, I64]),
             "nvfp4_gemm": (I, [P, P, P, P, P, P, P, I, I64, I64, I64, I64, P, SZ, P]),
+            "nvfp4_linear_workspace_bytes": (SZ, [I64, I64, I64]),
+            "nvfp4_linear": (I, [P, I64, I64, I64, P, P, P, P, I64, P, I, I64, P, SZ, P]),
             "nvfp4_gemm_swiglu_quant": (I, [P, P, P, P, P, P, P, P, P, I64, I64, I64, P]),
             "nvfp4_fuse_group_scales": (I, [I, P, I64, P, P, P, P, P]),
             "nvfp4_silu_mul": (I, [P, I64, I64, I64, P, I64, P]),
@@ -296,7 +299,41 @@ def read_fault(stream: torch.cuda.Stream | None = None) -> int:
     return int(v.value)
 
 
-def linear(x: torch.Tensor, w: NVFP4Tensor, out_dtype=torch.bfloat16,
+def linear_workspace_bytes(m: int, n: int, k: int) -> int:
+    return int(lib().nvfp4_linear_workspace_bytes(m, n, k))
+
+
+def linear_workspace(m: int, n: int, k: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace for linear() at these sizes (keep it: calls
+    leave the bytes that must start at zero zeroed again)."""
+    return torch.zeros(linear_workspace_bytes(m, n, k), dtype=torch.uint8, device=device)
+
+
+def linear(x: torch.Tensor, w: NVFP4Tensor, out: torch.Tensor | None = None,
+           out_dtype: torch.dtype = torch.bfloat16, global_scale: torch.Tensor | None = None,
+           workspace: torch.Tensor | None = None,
            stream: torch.cuda.Stream | None = None) -> torch.Tensor:
-    """The W4A4 linear layer: quantize x on the fly, then the FP4 GEMM."""
-    return gemm(quantize(x, stream=stream), w, out_dtype=out_dtype, stream=stream)
+    """nvfp4_linear, the W4A4 linear layer in one call: quantize x (dynamic
+    global, or the static ``global_scale``) and multiply with the NVFP4
+    weights ``w`` [n, k]; the GEMM's launch overlaps the quantization.
+    ``workspace`` from linear_workspace() (allocated here when None)."""
+    _require_cuda(x, "x", torch.bfloat16)
+    if x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be 2-D with unit stride along k")
+    m, k = x.shape
+    if k != w.k:
+        raise ValueError("k mismatch")
+    n = w.rows
+    if out is None:
+        out = torch.empty((m, n), dtype=out_dtype, device=x.device)
+    if out.dtype not in (torch.bfloat16, torch.float32) or out.stride(1) != 1:
+        raise ValueError("out must be bf16/fp32 with unit column stride")
+    if workspace is None:
+        workspace = linear_workspace(m, n, k, x.device)
+    st = lib().nvfp4_linear(_ptr(x), m, k, x.stride(0), _ptr(global_scale), _ptr(w.codes),
+                            _ptr(w.sf), _ptr(w.global_scale), n, _ptr(out),
+                            0 if out.dtype == torch.bfloat16 else 1, out.stride(0),
+                            _ptr(workspace), workspace.numel() * workspace.element_size(),
+                            _stream(stream))
+    _check(st, "nvfp4_linear")
+    return out

@@ -141,3 +141,34 @@ def test_swiglu_quant_argument_checks(L):
     assert f(*args(k=48)) == UNSUPPORTED
     assert f(*args(h=FAKE + 8)) == MISALIGNED
     assert f(*args(h=None)) == INVALID
+
+
+def lin(L, x=FAKE, m=8, k=64, ldx=64, xg=None, wc=FAKE, wsf=FAKE, wg=FAKE, n=64, y=FAKE, yd=0,
+        ldy=64, ws=FAKE, wsb=1 << 24):
+    return L.nvfp4_linear(P(x), m, k, ldx, P(xg), P(wc), P(wsf), P(wg), n, P(y), yd, ldy, P(ws),
+                          wsb, None)
+
+
+def test_linear_argument_checks(L):
+    assert lin(L, x=None) == INVALID
+    assert lin(L, ws=None) == INVALID
+    assert lin(L, m=0) == INVALID
+    assert lin(L, ldx=32) == INVALID         # ldx < k
+    assert lin(L, yd=2) == INVALID
+    assert lin(L, k=48, ldx=48) == UNSUPPORTED
+    assert lin(L, ws=FAKE + 16) == MISALIGNED  # workspace needs 256-byte alignment
+    assert lin(L, x=FAKE + 8) == MISALIGNED
+    assert lin(L, ldx=68) == MISALIGNED      # row pitch of x: 8 elements
+    assert lin(L, xg=FAKE + 2) == MISALIGNED
+    assert lin(L, wsb=16) == INVALID         # short workspace
+
+
+def test_linear_workspace_bytes(L):
+    f = L.nvfp4_linear_workspace_bytes
+    assert f(0, 64, 64) == 0 and f(8, 0, 64) == 0 and f(8, 64, 48) == 0
+    m, n, k = 8, 1000, 2048
+    # quantized activations + partial maxima + (few tokens) split counters and 8 slabs
+    assert f(m, n, k) >= m * k // 2 + L.nvfp4_sf_bytes(m, k) + 16384 + 8 * m * n * 4
+    assert f(65, n, k) < f(64, n, k)         # no split workspace above 64 tokens
+    assert L.nvfp4_gemm_workspace_bytes(m, n, k) == 256 + 8 * m * n * 4
+    assert L.nvfp4_gemm_workspace_bytes(65, n, k) == 0

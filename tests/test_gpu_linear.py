@@ -1,0 +1,122 @@
+"""GPU tests of nvfp4_linear, the W4A4 linear layer in one call (news article
+"Qwen3.8-27B最激进4bit量化开源…" §02: activations quantized to NVFP4 on the fly,
+then the GEMM on the 4-bit tensor cores), and of the few-token GEMM's split-K
+reduction.
+
+nvfp4_linear must equal nvfp4_quantize followed by nvfp4_gemm bit for bit (it
+runs the same kernels, only launched to overlap), and both agree with the
+oracle within the GEMM tolerance (parity.py). Weights come from the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity import bits, gemm_check, norms, upload
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    from nvfp4_w4a4_quantized_elem_b200 import build, nvfp4
+    build.build()
+    return nvfp4
+
+
+def gaussian(rows, k, seed, sigma=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn((rows, k), generator=g) * sigma).to(torch.bfloat16)
+
+
+def counter_bytes(n):
+    """Split counters at the start of the few-token workspace: 16 bytes per
+    128 weight rows, rounded up to 256 (nvfp4.h)."""
+    return -(-(16 * -(-n // 128)) // 256) * 256
+
+
+@pytest.mark.parametrize("m", [1, 16, 33, 64, 65, 300])
+@pytest.mark.parametrize("static", [False, True])
+def test_linear_equals_quantize_then_gemm(nv, orc, m, static):
+    k, n = 2048, 1000  # 8 weight tiles: few-token calls split K across the GPU
+    x = gaussian(m, k, 100 + m)
+    qw = orc.quantize(bits(gaussian(n, k, 5, 0.02)))
+    W = upload(qw)
+    xd = x.cuda()
+    g = None
+    if static:
+        # a static global from a calibration that saw a larger amax
+        g = torch.tensor([float(orc.global_from_amax(orc.tensor_amax(bits(x)) * 1.5))],
+                         dtype=torch.float32, device="cuda")
+    ws = nv.linear_workspace(m, n, k)
+    gws = torch.empty(max(16, nv.gemm_workspace_bytes(m, n, k)), dtype=torch.uint8,
+                      device="cuda")
+    qx = orc.quantize(bits(x), None if g is None else np.float32(g.item()))
+    ref = orc.gemm(qx, qw)
+    for dt in (torch.bfloat16, torch.float32):
+        y = nv.linear(xd, W, out_dtype=dt, global_scale=g, workspace=ws)
+        A = nv.quantize(xd, global_scale=g)
+        y2 = nv.gemm(A, W, out_dtype=dt, workspace=gws if m <= 64 else None)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y2), f"m={m} static={static} {dt}: linear != quantize + gemm"
+        gemm_check(y, ref, norms(orc, qx), norms(orc, qw), f"linear m={m} static={static} {dt}")
+    if m <= 64:
+        assert int(ws[:counter_bytes(n)].count_nonzero()) == 0, "split counters not reset"
+    assert nv.read_fault() == 0
+
+
+@pytest.mark.parametrize("m", [1, 32])
+def test_split_k_is_deterministic(nv, m):
+    """Decode shape 17408 -> 5120 (40 weight tiles, K in 3 slices): repeated
+    calls give identical bits, and the counters are zero afterwards."""
+    k, n = 17408, 5120
+    x = gaussian(m, k, 9).cuda()
+    W = nv.quantize(gaussian(n, k, 10, 0.02).cuda())
+    ws = nv.linear_workspace(m, n, k)
+    ys = [nv.linear(x, W, workspace=ws).clone() for _ in range(3)]
+    gws = torch.empty(nv.gemm_workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    A = nv.quantize(x)
+    gs = [nv.gemm(A, W, workspace=gws).clone() for _ in range(3)]
+    torch.cuda.synchronize()
+    for y in ys[1:] + gs:
+        assert torch.equal(y, ys[0])
+    assert int(ws[:counter_bytes(n)].count_nonzero()) == 0
+    assert int(gws[:counter_bytes(n)].count_nonzero()) == 0
+    assert nv.read_fault() == 0
+
+
+def test_linear_graph_replay(nv):
+    """A decode step captured once as a CUDA graph and replayed with new
+    activations written into the same input buffer gives the eager result."""
+    m, k, n = 1, 5120, 17408
+    W = nv.quantize(gaussian(n, k, 3, 0.02).cuda())
+    x = gaussian(m, k, 4).cuda()
+    y = torch.empty((m, n), dtype=torch.bfloat16, device="cuda")
+    ws = nv.linear_workspace(m, n, k)
+    nv.linear(x, W, out=y, workspace=ws)  # first call on the device outside the capture
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        nv.linear(x, W, out=y, workspace=ws)
+    for seed in (4, 5, 6):
+        x.copy_(gaussian(m, k, seed).cuda())
+        g.replay()
+        torch.cuda.synchronize()
+        ref = nv.linear(x, W, workspace=nv.linear_workspace(m, n, k))
+        torch.cuda.synchronize()
+        assert torch.equal(y, ref), f"graph replay differs for input seed {seed}"
+    assert nv.read_fault() == 0
+
+
+def test_linear_decode_full_size_against_oracle(nv, orc):
+    """The decode configuration at full size, sampled output columns against
+    the oracle (weights from the oracle, activations quantized on the GPU)."""
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+    cfg = wl.decode(8, 17408, 5120)
+    x = cfg.x()
+    qw = orc.quantize(bits(cfg.w()))
+    y = nv.linear(x.cuda(), upload(qw))
+    torch.cuda.synchronize()
+    qx = orc.quantize(bits(x))
+    ref = orc.gemm(qx, qw)
+    gemm_check(y, ref, norms(orc, qx), norms(orc, qw), "decode 8x17408->5120")
+    assert nv.read_fault() == 0
