@@ -149,3 +149,44 @@ DECODE_KN = ((5120, 17408), (17408, 5120))
 def decode(m: int, k: int, n: int) -> Linear:
     """Decode-shaped skinny GEMM: M tokens, weights [n, k] ~N(0,0.02)."""
     return Linear(f"decode_m{m}_k{k}_n{n}", m=m, n=n, k=k)
+
+
+@dataclass
+class Gates:
+    """The GDN gate projections a and b (48 heads each, the gdn_fused group's
+    modules: W_a ~N(0,0.1), W_b ~N(0,0.005)) on X ~N(0,1), with per-head gate
+    parameters drawn the way Gated DeltaNet layers are initialised:
+    A = exp(A_log) ~ U(1, 16) and dt ~ log-uniform on [1e-3, 1e-1] with
+    dt_bias = softplus^-1(dt) = log(expm1(dt)). FP64 parameters, seeds 5, 6."""
+    name: str = "gates"
+    m: int = 8192
+    k: int = 5120
+    heads: int = 48
+
+    def x(self, rows: int | None = None) -> torch.Tensor:
+        t = gaussian_bf16(self.m, self.k, 1.0, SEED_X)
+        return t if rows is None else t[:rows].contiguous()
+
+    def w_a(self, sigma: float = 0.1) -> torch.Tensor:
+        """sigma 0.1 as in the gdn_fused group; smaller values give the O(1)
+        gate pre-activations of a trained layer."""
+        return gaussian_bf16(self.heads, self.k, sigma, 3)
+
+    def w_b(self) -> torch.Tensor:
+        return gaussian_bf16(self.heads, self.k, 0.005, 4)
+
+    def a_log(self) -> torch.Tensor:
+        g = torch.Generator().manual_seed(5)
+        return torch.log(1.0 + 15.0 * torch.rand(self.heads, generator=g, dtype=torch.float64))
+
+    def dt_bias(self) -> torch.Tensor:
+        g = torch.Generator().manual_seed(6)
+        u = torch.rand(self.heads, generator=g, dtype=torch.float64)
+        dt = torch.exp(torch.log(torch.tensor(1e-3, dtype=torch.float64)) +
+                       u * (torch.log(torch.tensor(1e-1, dtype=torch.float64)) -
+                            torch.log(torch.tensor(1e-3, dtype=torch.float64))))
+        return torch.log(torch.expm1(dt))
+
+
+def gates() -> Gates:
+    return Gates()

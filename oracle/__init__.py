@@ -290,3 +290,46 @@ def silu_mul(y) -> np.ndarray:
     out = np.empty((m, n), np.uint16)
     _load().orc_silu_mul(_ptr(yb), m, n, n2, _ptr(out))
     return out
+
+
+# -------------------------------------------------------------- GDN gates --
+# Reading of news article §01 (Gated DeltaNet 基础: the gates are parameterized
+# in log space; the formula itself was lost from the page) together with the
+# abstract's "softplus/exponential and sigmoid parameterizations": per head,
+#   g     = -exp(A_log) * softplus(a + dt_bias)   (log-space decay)
+#   alpha = exp(g)                                (forget gate)
+#   beta  = sigmoid(b)                            (write strength)
+# where a, b are the outputs of the a and b projections.
+
+def softplus(z):
+    z = np.asarray(z, dtype=np.float64)
+    return np.maximum(z, 0.0) + np.log1p(np.exp(-np.abs(z)))
+
+
+def sigmoid(z):
+    z = np.asarray(z, dtype=np.float64)
+    e = np.exp(-np.abs(z))
+    return np.where(z >= 0, 1.0 / (1.0 + e), e / (1.0 + e))
+
+
+def gdn_gates(y_a, y_b, a_log, dt_bias):
+    """(g, alpha, beta) in FP64 from projection outputs [tokens, heads]."""
+    g = -np.exp(np.asarray(a_log, np.float64)) * softplus(
+        np.asarray(y_a, np.float64) + np.asarray(dt_bias, np.float64))
+    return g, np.exp(g), sigmoid(y_b)
+
+
+def rel_fro(approx, exact) -> float:
+    approx = np.asarray(approx, np.float64)
+    exact = np.asarray(exact, np.float64)
+    return float(np.linalg.norm(approx - exact) / np.linalg.norm(exact))
+
+
+def gate_sensitivity(y_a_ref, y_b_ref, y_a, y_b, a_log, dt_bias) -> dict:
+    """Relative Frobenius errors of the projections and of the gates computed
+    from them (abstract and paper reading §4.2 (ii): the gate nonlinearities
+    compress the W4A4 GEMM error)."""
+    g0, al0, be0 = gdn_gates(y_a_ref, y_b_ref, a_log, dt_bias)
+    g1, al1, be1 = gdn_gates(y_a, y_b, a_log, dt_bias)
+    return {"gemm_a": rel_fro(y_a, y_a_ref), "gemm_b": rel_fro(y_b, y_b_ref),
+            "g": rel_fro(g1, g0), "alpha": rel_fro(al1, al0), "beta": rel_fro(be1, be0)}
