@@ -295,19 +295,27 @@ class Step:
         return self.y
 
 
-def gemm_source_hash() -> str:
-    p = os.path.join(ROOT, "nvfp4_w4a4_quantized_elem_b200", "csrc", "gemm_sm100.cuh")
-    return hashlib.sha256(open(p, "rb").read()).hexdigest()[:16]
+def kernel_source_hash() -> str:
+    """Hash of every kernel source: a DRAM-traffic figure is only reported
+    while the kernels are the ones it was measured on."""
+    d = os.path.join(ROOT, "nvfp4_w4a4_quantized_elem_b200", "csrc")
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(d)):
+        if f.endswith((".cu", ".cuh")):
+            h.update(f.encode())
+            h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def dram_traffic(workload: str):
-    """DRAM bytes per GEMM launch from the committed ncu summary, if it was
-    taken on the current GEMM source; else None."""
-    p = os.path.join(ROOT, "profiles", "gemm_traffic.json")
+    """DRAM bytes per launch of the roofline's kernel (per step for decode)
+    from the committed ncu summary, if it was taken on the current kernel
+    sources; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         d = json.load(open(p))
         e = d.get(workload)
-        if e and e.get("gemm_source_sha256_16") == gemm_source_hash():
+        if e and e.get("csrc_sha256_16") == kernel_source_hash():
             return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
