@@ -33,6 +33,8 @@ struct DeviceState {
   int sms = 0;
   bool gemm_smem_set = false;
   unsigned skinny_smem_set = 0;       // bit per token-tile instantiation
+  int amax_per_sm = 0;                // resident CTAs per SM of the quantizer's kernels
+  int quant_per_sm = 0;
   float* noalloc_partials = nullptr;  // device address of g_noalloc_partials
 };
 
@@ -132,16 +134,38 @@ size_t skinny_workspace_bytes(int64_t m, int64_t n) {
                                        sizeof(float);
 }
 
+// Resident CTAs per SM of the quantizer's two kernels (occupancy query, once
+// per device): their grids are capped at one full wave, since a partial
+// second wave of these streaming kernels ran with idle SMs.
+nvfp4_status quant_occupancy(DeviceState* st) {
+  using namespace nvfp4::quant;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  if (st->amax_per_sm == 0) {
+    int a = 0, q = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&a, amax_kernel, kAmaxThreads, 0) !=
+            cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&q, quantize_kernel, kQuantThreads, 0) !=
+            cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    st->amax_per_sm = a < 1 ? 1 : a;
+    st->quant_per_sm = q < 1 ? 1 : q;
+  }
+  return NVFP4_OK;
+}
+
 // CTAs of the amax pass: enough that every thread streams ~8 16-byte chunks
 // (the contiguous path is flat over elements, the strided one a warp per
-// row), at most 2 per SM. Sizing by rows alone starved few-row inputs.
-int64_t amax_blocks(int64_t rows, int64_t k, int64_t ldx, int sms) {
+// row), at most one resident wave. Sizing by rows alone starved few-row
+// inputs.
+int64_t amax_blocks(int64_t rows, int64_t k, int64_t ldx, const DeviceState* st) {
   using namespace nvfp4::quant;
   const int64_t per_block = (ldx == k) ? static_cast<int64_t>(kAmaxThreads) * 8 * 8
                                        : static_cast<int64_t>(kAmaxThreads / 32);
   const int64_t units = (ldx == k) ? rows * k : rows;
   int64_t blocks = ceil_div(units, per_block);
-  const int64_t cap = static_cast<int64_t>(sms) * kAmaxBlocksPerSM;
+  const int64_t cap = static_cast<int64_t>(st->sms) * st->amax_per_sm;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return blocks;
@@ -173,11 +197,14 @@ nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
 nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx,
                              const float* global_in, uint8_t* codes, uint8_t* sf,
                              float* global_out, float* partials, int64_t max_parts,
-                             const DeviceState* st, cudaStream_t s) {
+                             DeviceState* st, cudaStream_t s) {
   using namespace nvfp4::quant;
+  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
+  if (n_tasks >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;  // 32-bit task index
+  if (nvfp4_status e = quant_occupancy(st)) return e;
   int nparts = 0;
   if (global_in == nullptr) {
-    const int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
+    const int64_t blocks = amax_blocks(rows, k, ldx, st);
     if (blocks > max_parts) return NVFP4_ERR_UNSUPPORTED;
     nparts = static_cast<int>(blocks);
     amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
@@ -195,9 +222,8 @@ nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx
   a.codes = codes;
   a.sf = sf;
   a.global_out = global_out;
-  const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
   int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
-  const int64_t cap = static_cast<int64_t>(st->sms) * kQuantBlocksPerSM;
+  const int64_t cap = static_cast<int64_t>(st->sms) * st->quant_per_sm;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return launch_pdl(quantize_kernel, static_cast<unsigned>(blocks), kQuantThreads, 0, s, 1u, a);
@@ -293,7 +319,8 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k, int6
   DeviceState* st;
   if (nvfp4_status e = current_device(&dev, &st)) return e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  int64_t blocks = amax_blocks(rows, k, ldx, st->sms);
+  if (nvfp4_status e = quant_occupancy(st)) return e;
+  int64_t blocks = amax_blocks(rows, k, ldx, st);
   if (blocks > kMaxPartials) blocks = kMaxPartials;
   amax_kernel<<<static_cast<unsigned>(blocks), kAmaxThreads, 0, s>>>(
       static_cast<const uint16_t*>(x), rows, k, ldx, static_cast<float*>(workspace));
