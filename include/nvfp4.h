@@ -322,6 +322,19 @@ nvfp4_status nvfp4_silu_mul(const void* y, int64_t m, int64_t n, int64_t ldy,
  */
 nvfp4_status nvfp4_read_fault(nvfp4_stream_t stream, uint32_t* fault_out);
 
+/*
+ * nvfp4_selftest_wait_timeout — a diagnostic with no counterpart on the
+ * pages: checks on the GPU that a bounded wait gives up. One thread waits,
+ * with the same bounded-wait routine as the few-token GEMM's roles, on an
+ * mbarrier that nothing arrives at; after limit_ns nanoseconds (global timer)
+ * it records bit 256 in the fault word and the kernel returns. A following
+ * nvfp4_read_fault reports NVFP4_ERR_TIMEOUT with that bit set; the context
+ * stays usable.
+ *   limit_ns  1000 .. 10^10 (1 us .. 10 s).
+ * Errors: INVALID_ARG (limit out of range), CUDA.
+ */
+nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, nvfp4_stream_t stream);
+
 #ifdef __cplusplus
 }  /* extern "C" */
 #endif

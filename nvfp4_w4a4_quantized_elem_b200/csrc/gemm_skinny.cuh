@@ -99,13 +99,14 @@ struct Params {
 };
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
-                                             volatile uint32_t* abort_flag, uint32_t who) {
+                                             volatile uint32_t* abort_flag, uint32_t who,
+                                             uint64_t limit_ns = kWaitLimitNs) {
   if (ptx::mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
   while (true) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (ptx::globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1u;
       atomicOr(&g_fault_word, who);
       return false;
@@ -447,6 +448,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     __syncwarp();
     ptx::tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Self-test of the bounded wait every role of this kernel uses: one thread
+// waits on an mbarrier that nothing arrives at, with a caller-given limit;
+// the wait gives up, records kFaultSelftest in the fault word and the kernel
+// returns normally, leaving the context usable.
+enum : uint32_t { kFaultSelftest = 256u };
+
+__global__ void __launch_bounds__(32, 1) selftest_wait_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ uint32_t abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0u;
+    ptx::fence_mbarrier_init();
+    wait_bounded(&bar, 0u, &abort_flag, kFaultSelftest, limit_ns);  // phase 0 never completes
   }
 }
 

@@ -726,6 +726,13 @@ nvfp4_status nvfp4_silu_mul(const void* y, int64_t m, int64_t n, int64_t ldy, vo
   return launch_status();
 }
 
+nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, nvfp4_stream_t stream) {
+  if (limit_ns < 1000u || limit_ns > 10000000000ull) return NVFP4_ERR_INVALID_ARG;
+  nvfp4::skinny::selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      limit_ns);
+  return launch_status();
+}
+
 nvfp4_status nvfp4_read_fault(nvfp4_stream_t stream, uint32_t* fault_out) {
   if (fault_out == nullptr) return NVFP4_ERR_INVALID_ARG;
   unsigned int v = 0;

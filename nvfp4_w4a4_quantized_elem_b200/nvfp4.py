@@ -27,7 +27,8 @@ EXPORTS = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_quantize_workspace_by
            "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_calibrate_global",
            "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_linear_workspace_bytes",
            "nvfp4_linear", "nvfp4_gemm_swiglu_quant",
-           "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault")
+           "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault",
+           "nvfp4_selftest_wait_timeout")
 
 _lib = None
 _lock = threading.Lock()
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "nvfp4_fuse_group_scales": (I, [I, P, I64, P, P, P, P, P]),
             "nvfp4_silu_mul": (I, [P, I64, I64, I64, P, I64, P]),
             "nvfp4_read_fault": (I, [P, U32P]),
+            "nvfp4_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -297,6 +299,14 @@ def read_fault(stream: torch.cuda.Stream | None = None) -> int:
     if st not in (NVFP4_OK, 5):
         raise NVFP4Error("nvfp4_read_fault", st)
     return int(v.value)
+
+
+def selftest_wait_timeout(limit_ns: int = 1_000_000,
+                          stream: torch.cuda.Stream | None = None) -> None:
+    """nvfp4_selftest_wait_timeout: make one bounded wait give up on the GPU
+    (read_fault() then returns 256)."""
+    _check(lib().nvfp4_selftest_wait_timeout(limit_ns, _stream(stream)),
+           "nvfp4_selftest_wait_timeout")
 
 
 def linear_workspace_bytes(m: int, n: int, k: int) -> int:

@@ -172,3 +172,10 @@ def test_linear_workspace_bytes(L):
     assert f(65, n, k) < f(64, n, k)         # no split workspace above 64 tokens
     assert L.nvfp4_gemm_workspace_bytes(m, n, k) == 256 + 8 * m * n * 4
     assert L.nvfp4_gemm_workspace_bytes(65, n, k) == 0
+
+
+def test_selftest_limit_checks(L):
+    f = L.nvfp4_selftest_wait_timeout
+    assert f(0, None) == INVALID
+    assert f(999, None) == INVALID
+    assert f(20_000_000_000, None) == INVALID
