@@ -427,6 +427,7 @@ def run_gpu(args):
     e2e["value"] = job_throughput(flops, world, e2e["ms_per_step"])
 
     assert nvfp4.read_fault(stream) == 0
+    lib_ref = cublaslt_reference(step, wk, stream, flush) if not wk.get("decode") else None
     traffic = dram_traffic(args.workload)
     if wk.get("decode"):
         # the whole layer per step: weights (codes + scales) once, X in bf16,
@@ -474,6 +475,8 @@ def run_gpu(args):
             "amax_gbs": round(amax_gbs, 1),
             "hbm_peak_gbs": pk["hbm_gbs"],
             "quant_bytes_per_elem": QUANT_BYTES_PER_ELEM,
+            "cublaslt_nvfp4_tflops": lib_ref,
+            "gemm_vs_cublaslt": (round(gemm_tflops / lib_ref, 4) if lib_ref else None),
         },
         "e2e": {"value": round(e2e["value"], 2), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
@@ -488,6 +491,43 @@ def run_gpu(args):
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def cublaslt_reference(step, wk, stream, flush, reps=20):
+    """The same first GEMM of the step through cuBLASLt's NVFP4 path
+    (torch._scaled_mm on the step's own codes and swizzled block scales; no
+    global scales, which do not change its time), L2 flushed before each
+    call: the library ceiling on this machine, reported as context. None where
+    this torch has no NVFP4 path."""
+    try:
+        if wk["kind"] == "linear":
+            B = wk["W"]
+        elif wk["kind"] == "mlp_fused":
+            B = wk["Wgi"]
+        else:
+            B = wk["Wgu"]
+        A = step.A
+        a = A.codes.view(torch.float4_e2m1fn_x2)
+        b = B.codes.view(torch.float4_e2m1fn_x2)
+        sa = A.sf.view(torch.float8_e4m3fn)
+        sb = B.sf.view(torch.float8_e4m3fn)
+        with torch.cuda.stream(stream):
+            f = lambda: torch._scaled_mm(a, b.t(), sa, sb, out_dtype=torch.bfloat16)
+            f()
+            evs = []
+            for _ in range(reps):
+                flush.fill_(7)
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                f()
+                e1.record(stream)
+                evs.append((e0, e1))
+        stream.synchronize()
+        ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in evs)
+        m, k = A.rows, A.k
+        return round(2 * m * B.rows * k / (ms * 1e-3) / 1e12, 1)
+    except Exception:
+        return None
 
 
 def separate_phases(step, wk, stream, flush, reps=20):
@@ -541,15 +581,22 @@ def measure_e2e(step, wk, stream, flops, args):
 
 # ------------------------------------------------------------ CPU oracle arm --
 
-def oracle_sample_step(orc, wk_cpu, rows):
+def oracle_sample_step(orc, wk_cpu, rows, times=None):
     """One bounded sample of the step on the CPU oracle: quantize `rows` rows
-    of X (dynamic global over the sample) and their FP64 GEMM rows."""
+    of X (dynamic global over the sample) and their FP64 GEMM rows. `times`
+    (a dict) accumulates the seconds spent quantizing X and in the GEMMs."""
     import numpy as np
     rows = min(rows, len(wk_cpu["x_bits"]))
     xs = wk_cpu["x_bits"][:rows]
+    t0 = time.perf_counter()
     qa = orc.quantize(np.ascontiguousarray(xs))
+    t1 = time.perf_counter()
     if wk_cpu["kind"] == "linear":
-        return orc.gemm(qa, wk_cpu["qw"])
+        y = orc.gemm(qa, wk_cpu["qw"])
+        if times is not None:
+            times["quant"] = times.get("quant", 0.0) + t1 - t0
+            times["gemm"] = times.get("gemm", 0.0) + time.perf_counter() - t1
+        return y
     y = orc.gemm(qa, wk_cpu["qgu"])
     yb = torch.from_numpy(y).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
     h = orc.silu_mul(yb)
@@ -593,22 +640,39 @@ def oracle_workload(name):
                      flops_per_row=2 * (2 * cfg.ffn) * cfg.d + 2 * cfg.d * cfg.ffn)
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def cpu_baseline(name, budget_s=15.0, rows=128):
     orc, w = oracle_workload(name)
     rows = min(rows, len(w["x_bits"]))
     oracle_sample_step(orc, w, 8)  # warm (builds/loads the oracle)
     t0 = time.perf_counter()
     reps = 0
+    times = {}
     while True:
-        oracle_sample_step(orc, w, rows)
+        oracle_sample_step(orc, w, rows, times)
         reps += 1
         el = time.perf_counter() - t0
         if el >= budget_s or reps >= 50:
             break
     tflops = w["flops_per_row"] * rows * reps / el / 1e12
-    return {"value": tflops, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
-            "sample": f"{reps} x ({rows} rows of X: oracle quantize + FP64 GEMM vs the full "
-                      f"pre-quantized weights), {el:.1f} s of host time, scaled per FLOP"}
+    out = {"value": tflops, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+           "cpu_model": cpu_model(),
+           "sample": f"{reps} x ({rows} rows of X: oracle quantize + FP64 GEMM vs the full "
+                     f"pre-quantized weights), {el:.1f} s of host time, scaled per FLOP"}
+    if times.get("quant"):
+        k = w["x_bits"].shape[1]
+        out["quant_gbs"] = round(reps * rows * k * QUANT_BYTES_PER_ELEM / times["quant"] / 1e9, 4)
+        out["gemm_gflops"] = round(w["flops_per_row"] * rows * reps / times["gemm"] / 1e9, 2)
+    return out
 
 
 def run_reference(args):
