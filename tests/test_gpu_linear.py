@@ -34,9 +34,11 @@ def counter_bytes(n):
     return -(-(16 * -(-n // 128)) // 256) * 256
 
 
-@pytest.mark.parametrize("m", [1, 16, 33, 64, 65, 300])
+@pytest.mark.parametrize("m", [1, 8, 16, 33, 64, 65, 300])
 @pytest.mark.parametrize("static", [False, True])
 def test_linear_equals_quantize_then_gemm(nv, orc, m, static):
+    """Few-token (m <= 64, K split) and paired (m > 64) GEMMs behind the
+    quantizer; the result is the two-call chain's."""
     k, n = 2048, 1000  # 8 weight tiles: few-token calls split K across the GPU
     x = gaussian(m, k, 100 + m)
     qw = orc.quantize(bits(gaussian(n, k, 5, 0.02)))
@@ -61,6 +63,22 @@ def test_linear_equals_quantize_then_gemm(nv, orc, m, static):
         gemm_check(y, ref, norms(orc, qx), norms(orc, qw), f"linear m={m} static={static} {dt}")
     if m <= 64:
         assert int(ws[:counter_bytes(n)].count_nonzero()) == 0, "split counters not reset"
+    assert nv.read_fault() == 0
+
+
+def test_linear_strided_and_ragged_x(nv, orc):
+    """x with a row pitch larger than k, and k not a multiple of 256 (the last
+    k-tile of every slice is partial): linear equals the chain."""
+    for m, k, n in [(3, 2080, 640), (40, 2080, 640), (1, 5152, 1000)]:
+        big = gaussian(m, k + 64, 21 + m).cuda()
+        x = big[:, :k]
+        W = nv.quantize(gaussian(n, k, 22, 0.02).cuda())
+        y = nv.linear(x, W)
+        gws = torch.empty(max(16, nv.gemm_workspace_bytes(m, n, k)), dtype=torch.uint8,
+                          device="cuda")
+        y2 = nv.gemm(nv.quantize(x), W, workspace=gws if m <= 64 else None)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y2), (m, k, n)
     assert nv.read_fault() == 0
 
 
