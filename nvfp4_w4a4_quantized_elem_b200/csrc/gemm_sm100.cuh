@@ -21,13 +21,20 @@
 //           one thread issues 4 MMAs (kind::mxf4nvf4.block16, K = 64) per
 //           256-element k-tile, then commits to the empty barrier of both
 //           CTAs and to the scale buffer's empty barrier.
-//   warps 2, 3  (even CTA) copy each stage's scale atoms into one of 4
-//           tensor-memory scale buffers (tcgen05.cp 32x128b.warpx4, both
-//           CTAs), 6 of the 12 copies each, and commit to that buffer's full
-//           barrier. Each tcgen05.cp costs a fixed ~50 cycles whatever its
-//           size; issued from the MMA thread the 12 copies per k-tile
-//           serialise with the 4 MMAs (about half the tensor-pipe time), and
-//           one copy warp alone issues slower than the MMAs consume.
+//   warps 2, 3  (even CTA) copy each stage's scale atoms into that stage's
+//           tensor-memory scale buffer (one per ring stage; tcgen05.cp
+//           32x128b.warpx4, both CTAs), 6 of the 12 copies each, and commit
+//           to the buffer's full barrier. Each tcgen05.cp costs a fixed ~50
+//           cycles whatever its size; issued from the MMA thread the 12 copies
+//           per k-tile serialise with the 4 MMAs (measured 4302 -> 2803 TF/s),
+//           and one copy warp alone issues slower than the MMAs consume.
+//           A buffer is reused only when its stage is refilled, which already
+//           waited for the stage's MMAs: the copy warps wait for nothing but
+//           the data, run ahead of the MMA thread, and their commits (which
+//           arrive only after the tensor work queued before them) are
+//           complete when the MMA thread needs them. A separate "buffer free"
+//           commit from the MMA thread made the copies trail the MMAs and
+//           drained the tensor pipe once per k-tile (~15%).
 //   warps 4..11  epilogue (both CTAs): two warps per tensor-memory lane
 //           quarter drain 128 columns each into registers, release the
 //           accumulator (arrive on the even CTA's barrier), then scale by
@@ -85,9 +92,10 @@ constexpr int EPI_WARP0 = SF_WARP0 + NUM_SF_WARPS;  // warps 4..11
 constexpr int NUM_THREADS = 32 * EPI_WARP0 + 32 * NUM_EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;               // [0, 256): FP32 accumulator
-constexpr int NSF = 4;                        // tensor-memory scale buffers
+constexpr int NSF = STAGES;                   // tensor-memory scale buffers, one per stage
 constexpr uint32_t SF_COL = 256;              // NSF x 48 columns: [A 16 | B 32]
 constexpr uint32_t SF_BUF_COLS = 48;
+static_assert(SF_COL + NSF * SF_BUF_COLS <= TMEM_COLS, "scale buffers exceed tensor memory");
 constexpr int GROUP_M = 16;                   // raster: 16 M-tiles per band
 constexpr int EPI_CHUNK_BYTES = 32 * 64;      // 32 rows x 64 bytes, 64-byte swizzle
 constexpr int EPI_WARP_BYTES = 2 * EPI_CHUNK_BYTES;
@@ -285,8 +293,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
   uint64_t* sf_full = drain + 1;
-  uint64_t* sf_empty = sf_full + NSF;
-  uint64_t* drain_sf = sf_empty + NSF;
+  uint64_t* drain_sf = sf_full + NSF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
@@ -307,7 +314,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(drain, 1);
     for (int b = 0; b < NSF; ++b) {
       ptx::mbar_init(&sf_full[b], NUM_SF_WARPS);
-      ptx::mbar_init(&sf_empty[b], 1);
     }
     ptx::mbar_init(drain_sf, NUM_SF_WARPS);
     *abort_flag = 0u;
@@ -409,12 +415,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ----------------------------------------------------------- MMA issuer --
     if (leader && lane == 0) {
       const uint32_t smem_base = ptx::smem_u32(smem);
-      uint32_t stage = 0, phase = 0, acc_phase = 0, sf_buf = 0, sf_phase = 0;
+      uint32_t stage = 0, phase = 0, acc_phase = 0;
       bool aborted = false;
       for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
         for (int kt = 0; kt < p.num_k_tiles; ++kt) {
           if (!wait_bounded(&full[stage], phase, ab, kFaultMma) ||
-              !wait_bounded(&sf_full[sf_buf], sf_phase, ab, kFaultMma)) {
+              !wait_bounded(&sf_full[stage], phase, ab, kFaultMma)) {
             aborted = true;
             break;
           }
@@ -429,8 +435,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             ptx::tc_fence_after();
           }
-          const uint32_t tsfa = sfa_cols(tmem, sf_buf);
-          const uint32_t tsfb = sfb_cols(tmem, sf_buf);
+          const uint32_t tsfa = sfa_cols(tmem, stage);
+          const uint32_t tsfb = sfb_cols(tmem, stage);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint64_t adesc = ptx::smem_desc(sa + 32u * j, 16, 1024, 2);
@@ -438,12 +444,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_mma_nvf4_pair(tmem + ACC_COL, adesc, bdesc, IDESC, tsfa + 4u * j,
                                   tsfb + 8u * j, (kt | j) != 0 ? 1u : 0u);
           }
-          ptx::tc_commit_pair_mc(&empty[stage], 0x3);  // frees the stage in both CTAs
-          ptx::tc_commit_pair_mc(&sf_empty[sf_buf], 0x1);  // frees the scale buffer
-          if (++sf_buf == NSF) {
-            sf_buf = 0;
-            sf_phase ^= 1u;
-          }
+          // frees the stage in both CTAs, and with it the stage's scale buffer
+          ptx::tc_commit_pair_mc(&empty[stage], 0x3);
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -462,23 +464,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ----------------------------------------------------- scale-copy warps --
     if (leader && lane == 0) {
       const uint32_t smem_base = ptx::smem_u32(smem);
-      uint32_t stage = 0, phase = 0, sf_buf = 0, sf_phase = 0;
+      uint32_t stage = 0, phase = 0;
       bool aborted = false;
       for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
         for (int kt = 0; kt < p.num_k_tiles; ++kt) {
-          if (!wait_bounded(&full[stage], phase, ab, kFaultScales) ||
-              !wait_bounded(&sf_empty[sf_buf], sf_phase ^ 1u, ab, kFaultScales)) {
+          // The stage's data having landed also means the MMAs of its previous
+          // use finished (the producer waited for them before reloading it),
+          // so scale buffer `stage` is free: no wait on the MMA thread here.
+          if (!wait_bounded(&full[stage], phase, ab, kFaultScales)) {
             aborted = true;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t ssfa = smem_base + stage * STAGE_BYTES + A_BYTES + B_BYTES;
-          copy_scales(tmem, ssfa, ssfa + SFA_BYTES, sf_buf, warp - SF_WARP0);
-          ptx::tc_commit_pair_mc(&sf_full[sf_buf], 0x1);  // buffer ready when copies land
-          if (++sf_buf == NSF) {
-            sf_buf = 0;
-            sf_phase ^= 1u;
-          }
+          copy_scales(tmem, ssfa, ssfa + SFA_BYTES, stage, warp - SF_WARP0);
+          ptx::tc_commit_pair_mc(&sf_full[stage], 0x1);  // buffer ready when copies land
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
