@@ -213,10 +213,11 @@ def make_workload(name: str, rank: int):
 
 
 class Step:
-    """One pass of the hot path. Prefill workloads: the library calls with CUDA
-    events between the phases. Decode workloads: one nvfp4_linear call
-    (quantizer and GEMM overlapped, so no event can sit between them),
-    captured once as a CUDA graph and replayed."""
+    """One pass of the hot path. Linear workloads: one nvfp4_linear call (the
+    layer as a user calls it; its GEMM launch overlaps the quantizer, so no
+    event can sit between them); decode ones are captured once as a CUDA graph
+    and replayed. MLP workloads: the library calls with CUDA events between
+    the phases. Phase times of linear workloads come from separate_phases()."""
 
     def __init__(self, wk, stream):
         from nvfp4_w4a4_quantized_elem_b200 import nvfp4
@@ -247,6 +248,9 @@ class Step:
         if self.gws is not None:
             self.launches += 1  # split-counter clear of nvfp4_gemm
         self.graph = None
+        self.fused_call = wk["kind"] == "linear"
+        if self.fused_call:
+            self.lws = nvfp4.linear_workspace(m, wk["W"].rows, k, dev)
         if wk.get("decode"):
             self.launches = 3   # amax, quantizer, few-token GEMM (counters stay zero)
             self.lws = nvfp4.linear_workspace(m, wk["W"].rows, k, dev)
@@ -259,7 +263,7 @@ class Step:
             stream.synchronize()
 
     def phases(self) -> int:
-        if self.graph is not None:
+        if self.fused_call:
             return 2
         return {"linear": 3, "mlp": 5, "mlp_fused": 4}[self.wk["kind"]]
 
@@ -277,6 +281,10 @@ class Step:
             self.graph.replay()
             rec(1)
             return self.y
+        if self.fused_call:
+            nv.linear(x, wk["W"], out=y, workspace=self.lws, stream=s)
+            rec(1)
+            return y
         nv.quantize(x, out=self.A, workspace=self.ws, stream=s)
         rec(1)
         if wk["kind"] == "linear":
@@ -389,12 +397,15 @@ def run_gpu(args):
     clocks = sampler.summary(t0, t1)
 
     step_ms = [events[i][0].elapsed_time(events[i][nph - 1]) for i in range(args.steps)]
-    if step.graph is None:
+    if not step.fused_call:
         quant_ms = [events[i][0].elapsed_time(events[i][1]) for i in range(args.steps)]
         gemm_ms = [events[i][1].elapsed_time(events[i][2]) for i in range(args.steps)]
+        phase_timing = "CUDA events between the phases of the timed steps"
     else:
         # the overlapped call has no boundary to time: the phases alone, L2 flushed
         quant_ms, gemm_ms = separate_phases(step, wk, stream, flush)
+        phase_timing = ("quantizer and GEMM each launched alone after the timed steps, "
+                        "20 times, CUDA events on their stream, L2 flushed before each")
     total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / args.steps
     value = job_throughput(flops, world, ms_per_step)
@@ -471,6 +482,7 @@ def run_gpu(args):
                      "frac_of_fp4_spec_9000": round(gemm_tflops / FP4_SPEC_TFLOPS, 4),
                      "algorithmic_flops_per_launch": 2 * gemm0[0] * gemm0[1] * gemm0[2]},
         "components": {
+            "phase_timing": phase_timing,
             "quantize_ms": round(q_avg_ms, 5), "gemm_ms": round(gemm_avg_ms, 5),
             "quantizer_alone_ms": round(qstatic_ms, 5), "amax_ms_est": round(amax_ms, 5),
             "quant_gbs": round(quant_gbs, 1),
