@@ -26,10 +26,12 @@
 //              ring of up to 8 stages.
 //   warp 1     allocates tensor memory; one thread issues 4 MMAs
 //              (kind::mxf4nvf4.block16, M = 128, N = BNT, K = 64) per k-tile.
-//   warps 2-3  copy the stage's scale atoms into one of 4 tensor-memory scale
-//              buffers (tcgen05.cp 32x128b.warpx4, ~50 cycles each whatever
-//              the size): with only ~18 KiB of weights per k-tile the copies
-//              would otherwise set the pace of the weight stream.
+//   warps 2-3  copy the stage's scale atoms into that stage's tensor-memory
+//              scale buffer (tcgen05.cp 32x128b.warpx4, ~50 cycles each
+//              whatever the size): with only ~18 KiB of weights per k-tile
+//              the copies would otherwise set the pace of the weight stream.
+//              A buffer is reused only when its stage is refilled, so the
+//              copy warps wait for nothing but the data.
 //   warps 4-7  epilogue: each thread owns one weight row (= one output
 //              column n) and drains its BNT token values 32 at a time; for a
 //              fixed token the 32 lanes write 32 consecutive columns.
@@ -53,10 +55,8 @@ constexpr int BK_BYTES = BK / 2;
 constexpr int NUM_THREADS = 256;
 constexpr int SF_WARP0 = 2;       // warps 2, 3 copy scales
 constexpr int EPI_WARP0 = 4;      // warps 4..7 drain the accumulator
-constexpr int NSF = 4;            // tensor-memory scale buffers
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL = 256;  // NSF x 48 columns after the accumulator
-constexpr uint32_t SF_BUF_COLS = 48;
+constexpr uint32_t SF_BUF_COLS = 48;  // per scale buffer: weights 16, tokens up to 32
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 constexpr size_t kSmemBudget = 220 * 1024;
@@ -78,6 +78,10 @@ struct Cfg {
   static constexpr int STAGES_FIT = static_cast<int>(kSmemBudget / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
+  // one tensor-memory scale buffer per stage, after the BNT-column accumulator
+  static constexpr int NSF = STAGES;
+  static constexpr uint32_t SF_COL = BNT < 32 ? 32u : static_cast<uint32_t>(BNT);
+  static_assert(SF_COL + NSF * SF_BUF_COLS <= TMEM_COLS, "scale buffers exceed tensor memory");
   static constexpr uint32_t SFB_COLS = 4u * SFB_BLOCKS;     // per K = 64 step
   // kind::mxf4nvf4, E2M1 x E2M1, both K-major, N = BNT, UE4M3 scales, M = 128
   static constexpr uint32_t IDESC = (1u << 7) | (1u << 10) |
@@ -163,8 +167,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* tmem_empty = tmem_full + 1;
   uint64_t* drain = tmem_empty + 1;
   uint64_t* sf_full = drain + 1;
-  uint64_t* sf_empty = sf_full + NSF;
-  uint64_t* drain_sf = sf_empty + NSF;
+  uint64_t* drain_sf = sf_full + C::NSF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
 
@@ -178,9 +181,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::mbar_init(tmem_full, 1);
     ptx::mbar_init(tmem_empty, 4);
     ptx::mbar_init(drain, 1);
-    for (int b = 0; b < NSF; ++b) {
+    for (int b = 0; b < C::NSF; ++b) {
       ptx::mbar_init(&sf_full[b], 2);
-      ptx::mbar_init(&sf_empty[b], 1);
     }
     ptx::mbar_init(drain_sf, 2);
     *abort_flag = 0u;
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ----------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       const uint32_t smem_base = ptx::smem_u32(smem);
-      uint32_t stage = 0, phase = 0, acc_phase = 0, sf_buf = 0, sf_phase = 0;
+      uint32_t stage = 0, phase = 0, acc_phase = 0;
       bool aborted = false;
       for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
         const int sp = u / p.num_w_tiles;
@@ -271,14 +273,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tc_fence_after();
         for (int kt = k0; kt < k1; ++kt) {
           if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma) ||
-              !wait_bounded(&sf_full[sf_buf], sf_phase, abort_flag, kFaultMma)) {
+              !wait_bounded(&sf_full[stage], phase, abort_flag, kFaultMma)) {
             aborted = true;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t sa = smem_base + stage * C::STAGE_BYTES;
           const uint32_t sb = sa + C::A_BYTES;
-          const uint32_t tsfa = tmem + SF_COL + sf_buf * SF_BUF_COLS;
+          const uint32_t tsfa = tmem + C::SF_COL + stage * SF_BUF_COLS;
           const uint32_t tsfb = tsfa + 16u;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -287,12 +289,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             ptx::tc_mma_nvf4(tmem, adesc, bdesc, C::IDESC, tsfa + 4u * j, tsfb + C::SFB_COLS * j,
                              (kt != k0 || j != 0) ? 1u : 0u);
           }
-          ptx::tc_commit(&empty[stage]);
-          ptx::tc_commit(&sf_empty[sf_buf]);
-          if (++sf_buf == NSF) {
-            sf_buf = 0;
-            sf_phase ^= 1u;
-          }
+          ptx::tc_commit(&empty[stage]);  // frees the stage and its scale buffer
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -312,22 +309,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       const int part = warp - SF_WARP0;  // 0: weight scales, 1: token scales
       const uint32_t smem_base = ptx::smem_u32(smem);
-      uint32_t stage = 0, phase = 0, sf_buf = 0, sf_phase = 0;
+      uint32_t stage = 0, phase = 0;
       bool aborted = false;
       for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
         const int sp = u / p.num_w_tiles;
         const int k0 = sp * p.k_tiles_per_split;
         const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
         for (int kt = k0; kt < k1; ++kt) {
-          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales) ||
-              !wait_bounded(&sf_empty[sf_buf], sf_phase ^ 1u, abort_flag, kFaultScales)) {
+          // the stage's data having landed means its previous MMAs finished
+          // (the producer waited for them), so scale buffer `stage` is free
+          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales)) {
             aborted = true;
             break;
           }
           ptx::tc_fence_after();
           const uint32_t ssfa = smem_base + stage * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES;
           const uint32_t ssfb = ssfa + C::SFA_BYTES;
-          const uint32_t tsfa = tmem + SF_COL + sf_buf * SF_BUF_COLS;
+          const uint32_t tsfa = tmem + C::SF_COL + stage * SF_BUF_COLS;
           const uint32_t tsfb = tsfa + 16u;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
@@ -340,11 +338,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                           ptx::smem_desc(ssfb + 2048u * h + 512u * j, 0, 128, 0));
             }
           }
-          ptx::tc_commit(&sf_full[sf_buf]);
-          if (++sf_buf == NSF) {
-            sf_buf = 0;
-            sf_phase ^= 1u;
-          }
+          ptx::tc_commit(&sf_full[stage]);
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
