@@ -157,7 +157,7 @@ def job_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> flo
 def make_workload(name: str, rank: int):
     """Device-resident inputs and pre-quantized weights of one workload."""
     from nvfp4_w4a4_quantized_elem_b200 import nvfp4, workloads as wl
-    if name == "outlier":
+    if name in ("outlier", "outlier_static"):
         cfg = wl.outlier()
         cfg.x_seed = rank_x_seed(rank)
         x = cfg.x().cuda()
@@ -165,7 +165,17 @@ def make_workload(name: str, rank: int):
         gemms = [(cfg.m, cfg.n, cfg.k)]
         desc = (f"outlier: X {cfg.m}x{cfg.k} bf16 ~N(0,1) with 8 channels x50, "
                 f"W {cfg.n}x{cfg.k} ~N(0,0.02) NVFP4; quantize X + W4A4 GEMM -> bf16")
-        return dict(x=x, W=W, gemms=gemms, desc=desc, kind="linear", m=cfg.m, n=cfg.n, k=cfg.k)
+        out = dict(x=x, W=W, gemms=gemms, desc=desc, kind="linear", m=cfg.m, n=cfg.n, k=cfg.k)
+        if name == "outlier_static":
+            # the served recipe's static activation global: calibrated once on
+            # four other seeded batches of the same distribution (running amax)
+            cal = nvfp4.Calibrator()
+            for seed in (101, 102, 103, 104):
+                cfg.x_seed = seed
+                cal.observe(cfg.x().cuda())
+            out["x_global"] = cal.global_scale
+            out["desc"] = desc.replace("quantize X", "quantize X with a calibrated static global")
+        return out
     if name == "gdn_fused":
         cfg = wl.gdn_fused()
         x = wl.gaussian_bf16(cfg.m, cfg.k, 1.0, rank_x_seed(rank)).cuda()
@@ -245,6 +255,8 @@ class Step:
             self.H = nvfp4.NVFP4Tensor.empty(m, ffn, dev)
             self.y = torch.empty((m, wk["n"]), dtype=torch.bfloat16, device=dev)
         self.launches = {"linear": 3, "mlp": 9, "mlp_fused": 4}[wk["kind"]]
+        if wk.get("x_global") is not None:
+            self.launches -= 1  # static global: no amax pass
         if self.gws is not None:
             self.launches += 1  # split-counter clear of nvfp4_gemm
         self.graph = None
@@ -282,7 +294,8 @@ class Step:
             rec(1)
             return self.y
         if self.fused_call:
-            nv.linear(x, wk["W"], out=y, workspace=self.lws, stream=s)
+            nv.linear(x, wk["W"], out=y, global_scale=wk.get("x_global"), workspace=self.lws,
+                      stream=s)
             rec(1)
             return y
         nv.quantize(x, out=self.A, workspace=self.ws, stream=s)
@@ -552,7 +565,8 @@ def separate_phases(step, wk, stream, flush, reps=20):
     q, g = [], []
     with torch.cuda.stream(stream):
         for _ in range(reps):
-            for fn, out in ((lambda: nvfp4.quantize(wk["x"], out=step.A, workspace=step.ws,
+            for fn, out in ((lambda: nvfp4.quantize(wk["x"], global_scale=wk.get("x_global"),
+                                                    out=step.A, workspace=step.ws,
                                                     stream=stream), q),
                             (lambda: nvfp4.gemm(step.A, wk["W"], out=step.y, workspace=step.gws,
                                                 stream=stream), g)):
@@ -675,6 +689,8 @@ def oracle_name(workload: str) -> str:
         return "mlp32k"
     if workload.startswith("decode:"):
         return workload
+    if workload == "outlier_static":
+        return "outlier"
     return workload
 
 
@@ -781,7 +797,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="outlier",
-                    help="outlier | gdn_fused | mlp32k | mlp32k_fused | decode:M:K:N")
+                    help="outlier | outlier_static | gdn_fused | mlp32k | mlp32k_fused | decode:M:K:N")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
