@@ -161,10 +161,11 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k,
                                     nvfp4_stream_t stream);
 
 /* Workspace bytes nvfp4_gemm can use: for m <= 64, 16*ceil(n/128) bytes of
- * split counters (rounded up to 256) plus 8*m*n*4 bytes for up to 8 FP32
- * slabs of Y (few-token GEMMs split K across CTAs and add the slabs in a fixed
- * order); else 0. Passing less (or NULL) is allowed and only disables the
- * split. */
+ * reduction counters (rounded up to 256) plus ceil(n/128)*9*m*128*4 bytes of
+ * FP32 partial slabs: with fewer 128-row weight tiles than SMs, few-token
+ * GEMMs deal the (tile, k-tile) iterations out to every SM in equal
+ * contiguous shares (stream-K) and add the partial tiles in a fixed order;
+ * else 0. Passing less (or NULL) is allowed and only disables the split. */
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -187,7 +188,7 @@ size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              (the call zeroes the split counters itself).
  * m <= 64 runs the few-token kernel (weights on the MMA's 128-row side,
  * tokens as its N); larger m the paired-CTA 256x256-tile kernel. Results do
- * not depend on the run: split-K slices are summed in slice order.
+ * not depend on the run: partial tiles are summed in k order.
  * The kernel is launched with programmatic stream serialisation; it reads and
  * writes global memory only after the previous kernel in the stream finished.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.

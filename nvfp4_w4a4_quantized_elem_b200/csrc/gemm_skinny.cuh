@@ -8,14 +8,17 @@
 // (W4A4 on 4-bit tensor cores); decode throughput is one of the serving
 // numbers the pages report (§04).
 //
-// One CTA per SM, persistent over work units (128 weight rows x one slice of
-// K). When the weight tiles alone cannot occupy the GPU, K is split across
-// CTAs (at most kMaxSplits slices): each slice writes its FP32 partial
-// (already scaled by 1/(g_a g_b)) to its own workspace slab; then each
-// epilogue warp counts itself in on the counter of its 32 output columns,
-// and the warp that arrives last for those columns sums the slabs in slice
-// order, writes Y and resets the counter. The result is the same on every
-// run, and no warp ever waits for another.
+// One CTA per SM. With at least as many weight tiles (128 rows each) as
+// CTAs, a CTA takes whole tiles. With fewer, the work is split stream-K
+// fashion: the W x KT (tile, k-tile) iterations are dealt out in G equal
+// contiguous shares, so every SM streams weights; a share may end inside one
+// tile and continue into the next. A segment that is only part of a tile
+// writes its FP32 partial (already scaled by 1/(g_a g_b)) to the slab of
+// its (tile, contributor) slot; then each epilogue warp counts itself in on
+// the counter of its 32 output columns, and the warp that arrives last for
+// those columns sums the tile's slabs in contributor (= k) order, writes Y
+// and resets the counter. The result is the same on every run, and no warp
+// ever waits for another.
 // Launched with programmatic stream serialisation: tensor-memory allocation
 // and barrier set-up overlap the previous kernel; every global access waits
 // for it, except that, when the caller guarantees the weights were written
@@ -60,8 +63,9 @@ constexpr uint32_t SF_BUF_COLS = 48;  // per scale buffer: weights 16, tokens up
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
 constexpr size_t kSmemBudget = 220 * 1024;
-constexpr int kMaxSplits = 8;     // K slices per weight tile
-constexpr int kSumTokens = 16;    // tokens summed per round of slab loads
+constexpr int kMaxSplits = 8;     // stream-K: at most this many CTAs per weight tile
+constexpr int kMaxContrib = kMaxSplits + 1;  // contributor slots per tile (host-checked)
+constexpr int kSumTokens = 8;     // tokens summed per round of slab loads
 
 enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, kFaultScales = 128u };
 
@@ -91,14 +95,15 @@ struct Cfg {
 
 struct Params {
   int M, N, K;              // Y is [M][N]; weights are [N][K], tokens [M][K]
-  int num_w_tiles, num_k_tiles, splits, k_tiles_per_split;
+  int num_w_tiles, num_k_tiles;
+  int stream_k;             // 1: contiguous shares of the tile x k-tile iterations
   const float* a_global;    // tokens' global
   const float* b_global;    // weights' global
   void* y;                  // direct mode: [M][ldy] bf16 / fp32
   int64_t ldy;
   int y_fp32;
-  float* partial;           // split mode: [splits][M][N] FP32 slabs
-  unsigned int* tile_count; // split mode: [num_w_tiles * 4], zero before and after a launch
+  float* partial;           // stream-K: [num_w_tiles][kMaxContrib][M][BW] FP32 slabs
+  unsigned int* tile_count; // stream-K: [num_w_tiles * 4], zero before and after a launch
   int early_w;              // weights may be read before the previous kernel finishes
 };
 
@@ -136,19 +141,62 @@ __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[3
       : "memory");
 }
 
-// Issue order of the producer: (unit, k-tile) pairs of this CTA.
-struct WorkIter {
-  int u, kt, k1, wt;
-  __device__ __forceinline__ void start(int unit, const Params& p, int num_units) {
-    u = unit;
-    if (u < num_units) {
-      wt = u % p.num_w_tiles;
-      kt = (u / p.num_w_tiles) * p.k_tiles_per_split;
-      k1 = min(p.num_k_tiles, kt + p.k_tiles_per_split);
+// The CTA that owns stream-K iteration `it` (shares are [c T / G, (c+1) T / G)).
+__device__ __forceinline__ int cta_of(int64_t it, int64_t T, int64_t G) {
+  return static_cast<int>(((it + 1) * G - 1) / T);
+}
+
+// This CTA's segments, in issue order: (weight tile, [k0, k1)).
+struct SegIter {
+  int64_t i, i1;  // stream-K: next iteration and end of this CTA's share
+  int wt, k0, k1;
+  bool valid;
+  __device__ __forceinline__ void load(const Params& p) {
+    valid = i < i1;
+    if (valid) {
+      wt = static_cast<int>(i / p.num_k_tiles);
+      k0 = static_cast<int>(i - static_cast<int64_t>(wt) * p.num_k_tiles);
+      k1 = static_cast<int>(min(static_cast<int64_t>(p.num_k_tiles), k0 + (i1 - i)));
     }
   }
-  __device__ __forceinline__ void next(const Params& p, int num_units) {
-    if (++kt >= k1) start(u + static_cast<int>(gridDim.x), p, num_units);
+  __device__ __forceinline__ void first(const Params& p) {
+    if (p.stream_k) {
+      const int64_t T = static_cast<int64_t>(p.num_w_tiles) * p.num_k_tiles;
+      const int64_t G = gridDim.x;
+      i = static_cast<int64_t>(blockIdx.x) * T / G;
+      i1 = (static_cast<int64_t>(blockIdx.x) + 1) * T / G;
+      load(p);
+    } else {
+      wt = blockIdx.x;
+      k0 = 0;
+      k1 = p.num_k_tiles;
+      valid = wt < p.num_w_tiles;
+    }
+  }
+  __device__ __forceinline__ void next(const Params& p) {
+    if (p.stream_k) {
+      i += k1 - k0;
+      load(p);
+    } else {
+      wt += gridDim.x;
+      valid = wt < p.num_w_tiles;
+    }
+  }
+};
+
+// Issue order of the producer: (segment, k-tile) pairs of this CTA.
+struct WorkIter {
+  SegIter sg;
+  int kt;
+  __device__ __forceinline__ void start(const Params& p) {
+    sg.first(p);
+    kt = sg.k0;
+  }
+  __device__ __forceinline__ void next(const Params& p) {
+    if (++kt >= sg.k1) {
+      sg.next(p);
+      kt = sg.k0;
+    }
   }
 };
 
@@ -200,7 +248,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const int num_units = p.num_w_tiles * p.splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
@@ -208,22 +255,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0;
       bool aborted = false;
       WorkIter it;
-      it.start(blockIdx.x, p, num_units);
+      it.start(p);
       // The first ring's worth of stages needs no empty-slot wait. With
       // early_w their weight halves are requested before the grid-dependency
       // wait, the token halves after it.
       int npre = 0;
       if (p.early_w) {
         WorkIter w = it;
-        for (; npre < C::STAGES && w.u < num_units; ++npre, w.next(p, num_units)) {
+        for (; npre < C::STAGES && w.sg.valid; ++npre, w.next(p)) {
           uint8_t* st = smem + npre * C::STAGE_BYTES;
           ptx::mbar_arrive_expect_tx(&full[npre], C::STAGE_RAW);
-          ptx::tma_load_2d(st, &tmW, &full[npre], w.kt * BK_BYTES, w.wt * BW);
-          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4, w.wt);
+          ptx::tma_load_2d(st, &tmW, &full[npre], w.kt * BK_BYTES, w.sg.wt * BW);
+          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4,
+                           w.sg.wt);
         }
       }
       ptx::grid_dep_wait();
-      for (int i = 0; i < npre; ++i, it.next(p, num_units)) {
+      for (int i = 0; i < npre; ++i, it.next(p)) {
         uint8_t* st = smem + i * C::STAGE_BYTES;
         ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[i], it.kt * BK_BYTES, 0);
         ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[i], 0,
@@ -232,7 +280,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       stage = static_cast<uint32_t>(npre % C::STAGES);
       phase = static_cast<uint32_t>(npre / C::STAGES);
-      for (; it.u < num_units; it.next(p, num_units)) {
+      for (; it.sg.valid; it.next(p)) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer)) {
           aborted = true;
           break;
@@ -240,9 +288,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         pending &= ~(1u << stage);
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
-        ptx::tma_load_2d(st, &tmW, &full[stage], it.kt * BK_BYTES, it.wt * BW);
+        ptx::tma_load_2d(st, &tmW, &full[stage], it.kt * BK_BYTES, it.sg.wt * BW);
         ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], it.kt * BK_BYTES, 0);
-        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, it.kt * 4, it.wt);
+        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, it.kt * 4,
+                         it.sg.wt);
         ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
                          it.kt * 4, 0);
         pending |= 1u << stage;
@@ -262,10 +311,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t smem_base = ptx::smem_u32(smem);
       uint32_t stage = 0, phase = 0, acc_phase = 0;
       bool aborted = false;
-      for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-        const int sp = u / p.num_w_tiles;
-        const int k0 = sp * p.k_tiles_per_split;
-        const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
+      SegIter sg;
+      for (sg.first(p); sg.valid && !aborted; sg.next(p)) {
+        const int k0 = sg.k0, k1 = sg.k1;
         if (!wait_bounded(tmem_empty, acc_phase ^ 1u, abort_flag, kFaultMma)) {
           aborted = true;
           break;
@@ -311,11 +359,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t smem_base = ptx::smem_u32(smem);
       uint32_t stage = 0, phase = 0;
       bool aborted = false;
-      for (int u = blockIdx.x; u < num_units && !aborted; u += gridDim.x) {
-        const int sp = u / p.num_w_tiles;
-        const int k0 = sp * p.k_tiles_per_split;
-        const int k1 = min(p.num_k_tiles, k0 + p.k_tiles_per_split);
-        for (int kt = k0; kt < k1; ++kt) {
+      SegIter sg;
+      for (sg.first(p); sg.valid && !aborted; sg.next(p)) {
+        for (int kt = sg.k0; kt < sg.k1; ++kt) {
           // the stage's data having landed means its previous MMAs finished
           // (the producer waited for them), so scale buffer `stage` is free
           if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales)) {
@@ -356,15 +402,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;  // tensor-memory lane quarter (warps 4..7 -> 0..3)
     const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
     uint32_t acc_phase = 0;
-    for (int u = blockIdx.x; u < num_units; u += gridDim.x) {
-      const int wt = u % p.num_w_tiles;
-      const int sp = u / p.num_w_tiles;
+    const int64_t T = static_cast<int64_t>(p.num_w_tiles) * p.num_k_tiles;
+    SegIter sg;
+    for (sg.first(p); sg.valid; sg.next(p)) {
+      const int wt = sg.wt;
+      const bool whole = sg.k0 == 0 && sg.k1 == p.num_k_tiles;  // no other contributor
+      int c_first = 0, n_contrib = 1;
+      if (!whole) {
+        c_first = cta_of(static_cast<int64_t>(wt) * p.num_k_tiles, T, gridDim.x);
+        n_contrib = cta_of(static_cast<int64_t>(wt + 1) * p.num_k_tiles - 1, T, gridDim.x) -
+                    c_first + 1;
+      }
       if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue)) break;
       ptx::tc_fence_after();
-      const int n = wt * BW + q * 32 + lane;   // this thread's output column
+      const int nl = q * 32 + lane;            // column within the weight tile
+      const int n = wt * BW + nl;              // this thread's output column
       const bool n_ok = n < p.N;
       const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
-      float* slab = p.splits > 1 ? p.partial + static_cast<int64_t>(sp) * p.M * p.N : nullptr;
+      // slab of this (tile, contributor): [M][BW]
+      float* slab = whole ? nullptr
+                          : p.partial + (static_cast<int64_t>(wt) * kMaxContrib +
+                                         (static_cast<int>(blockIdx.x) - c_first)) *
+                                            p.M * BW;
 #pragma unroll
       for (int c0 = 0; c0 < BNT; c0 += 32) {
         uint32_t r[32];
@@ -380,8 +439,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int m = c0 + i;                 // token
           if (m >= p.M || !n_ok) continue;
           const float v = __uint_as_float(r[i]) * alpha;
-          if (p.splits > 1) {
-            slab[static_cast<int64_t>(m) * p.N + n] = v;
+          if (!whole) {
+            slab[static_cast<int64_t>(m) * BW + nl] = v;
           } else if (p.y_fp32) {
             reinterpret_cast<float*>(p.y)[static_cast<int64_t>(m) * p.ldy + n] = v;
           } else {
@@ -394,34 +453,35 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(tmem_empty);
       acc_phase ^= 1u;
-      if (p.splits > 1) {
-        // count this slice in for these 32 columns; the last one sums them
+      if (!whole) {
+        // count this contributor in for these 32 columns; the last one sums
+        // the tile's slabs in contributor order (= k order)
         __threadfence();
         __syncwarp();
         uint32_t last = 0;
         if (lane == 0)
-          last = atomicAdd(p.tile_count + wt * 4 + q, 1u) == static_cast<unsigned>(p.splits - 1);
+          last = atomicAdd(p.tile_count + wt * 4 + q, 1u) == static_cast<unsigned>(n_contrib - 1);
         last = __shfl_sync(0xFFFFFFFFu, last, 0);
         if (last) {
           __threadfence();
           if (n_ok) {
+            const float* base = p.partial + static_cast<int64_t>(wt) * kMaxContrib * p.M * BW;
             for (int m0 = 0; m0 < p.M; m0 += kSumTokens) {
-              float v[kSumTokens][kMaxSplits];
+              float v[kSumTokens][kMaxContrib];
 #pragma unroll
               for (int i = 0; i < kSumTokens; ++i)
 #pragma unroll
-                for (int s2 = 0; s2 < kMaxSplits; ++s2)
-                  v[i][s2] = (s2 < p.splits && m0 + i < p.M)
-                                 ? __ldcg(p.partial + (static_cast<int64_t>(s2) * p.M + m0 + i) *
-                                                          p.N + n)
-                                 : 0.0f;
+                for (int j = 0; j < kMaxContrib; ++j)
+                  v[i][j] = (j < n_contrib && m0 + i < p.M)
+                                ? __ldcg(base + (static_cast<int64_t>(j) * p.M + m0 + i) * BW + nl)
+                                : 0.0f;
 #pragma unroll
               for (int i = 0; i < kSumTokens; ++i) {
                 if (m0 + i >= p.M) break;
                 float acc = v[i][0];
 #pragma unroll
-                for (int s2 = 1; s2 < kMaxSplits; ++s2)
-                  if (s2 < p.splits) acc += v[i][s2];
+                for (int j = 1; j < kMaxContrib; ++j)
+                  if (j < n_contrib) acc += v[i][j];
                 const int64_t o = static_cast<int64_t>(m0 + i) * p.ldy + n;
                 if (p.y_fp32)
                   reinterpret_cast<float*>(p.y)[o] = acc;

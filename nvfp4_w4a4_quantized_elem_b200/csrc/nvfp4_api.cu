@@ -123,15 +123,41 @@ nvfp4_status launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block,
   return NVFP4_OK;
 }
 
-// Few-token GEMM workspace: split counters (4 per 128 weight rows), then up
-// to kMaxSplits FP32 slabs of Y.
+// Few-token GEMM workspace: reduction counters (4 per 128 weight rows), then
+// kMaxContrib FP32 slabs of [m][128] per weight tile.
 size_t skinny_counter_bytes(int64_t n) {
   return round_up(static_cast<size_t>(ceil_div(n, 128)) * 4 * sizeof(unsigned int), 256);
 }
 size_t skinny_workspace_bytes(int64_t m, int64_t n) {
-  return skinny_counter_bytes(n) + static_cast<size_t>(nvfp4::skinny::kMaxSplits) *
-                                       static_cast<size_t>(m) * static_cast<size_t>(n) *
-                                       sizeof(float);
+  return skinny_counter_bytes(n) + static_cast<size_t>(ceil_div(n, 128)) *
+                                       nvfp4::skinny::kMaxContrib * static_cast<size_t>(m) *
+                                       nvfp4::skinny::BW * sizeof(float);
+}
+
+// Stream-K grid of a few-token GEMM: G CTAs sharing the W x KT iterations,
+// at most kMaxSplits per weight tile, shrunk until no tile has more than
+// kMaxContrib contributing CTAs (each has a slab slot). 0 = no split: whole
+// tiles, when they already occupy more than 3/4 of the SMs — the slab write
+// and in-order reduction of split tiles cost ~2 us, more than the extra SMs
+// bring then (measured: 136 tiles on 148 SMs, 24.2 -> 26.6 us per decode
+// step; 40 tiles, 30.8 -> 28.7 us).
+int skinny_stream_k_grid(int sms, int64_t w_tiles, int64_t k_tiles) {
+  using namespace nvfp4::skinny;
+  if (4 * w_tiles > 3 * static_cast<int64_t>(sms)) return 0;
+  const int64_t T = w_tiles * k_tiles;
+  int64_t G = sms;
+  if (G > T) G = T;
+  if (G > w_tiles * kMaxSplits) G = w_tiles * kMaxSplits;
+  auto owner = [&](int64_t it, int64_t g) { return ((it + 1) * g - 1) / T; };
+  for (; G > w_tiles; --G) {
+    int64_t worst = 0;
+    for (int64_t w = 0; w < w_tiles; ++w) {
+      const int64_t c = owner((w + 1) * k_tiles - 1, G) - owner(w * k_tiles, G) + 1;
+      if (c > worst) worst = c;
+    }
+    if (worst <= kMaxContrib) return static_cast<int>(G);
+  }
+  return 0;
 }
 
 // Resident CTAs per SM of the quantizer's two kernels (occupancy query, once
@@ -444,28 +470,25 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   p.partial = nullptr;
   p.tile_count = nullptr;
   p.early_w = early_w;
-  int splits = 1;
-  if (workspace != nullptr && workspace_bytes >= skinny_workspace_bytes(m, n) &&
-      aligned(workspace, 16)) {
-    splits = st->sms / p.num_w_tiles;
-    if (splits > p.num_k_tiles) splits = p.num_k_tiles;
-    if (splits > kMaxSplits) splits = kMaxSplits;
-    if (splits < 1) splits = 1;
-  }
-  p.k_tiles_per_split = static_cast<int>(ceil_div(p.num_k_tiles, splits));
-  splits = static_cast<int>(ceil_div(p.num_k_tiles, p.k_tiles_per_split));  // no empty slice
-  p.splits = splits;
-  if (splits > 1) {
-    p.tile_count = static_cast<unsigned int*>(workspace);
-    p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                         skinny_counter_bytes(n));
-    if (zero_counters && cudaMemsetAsync(workspace, 0, skinny_counter_bytes(n), s) != cudaSuccess) {
-      cudaGetLastError();
-      return NVFP4_ERR_CUDA;
+  p.stream_k = 0;
+  int grid = static_cast<int>(p.num_w_tiles < st->sms ? p.num_w_tiles : st->sms);
+  const bool split_ok = workspace != nullptr &&
+                        workspace_bytes >= skinny_workspace_bytes(m, n) && aligned(workspace, 16);
+  if (split_ok) {
+    const int g = skinny_stream_k_grid(st->sms, p.num_w_tiles, p.num_k_tiles);
+    if (g > 0) {
+      p.stream_k = 1;
+      grid = g;
+      p.tile_count = static_cast<unsigned int*>(workspace);
+      p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           skinny_counter_bytes(n));
+      if (zero_counters &&
+          cudaMemsetAsync(workspace, 0, skinny_counter_bytes(n), s) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+      }
     }
   }
-  const int64_t units = static_cast<int64_t>(p.num_w_tiles) * splits;
-  const int grid = static_cast<int>(units < st->sms ? units : st->sms);
   nvfp4_status e;
   switch (bnt) {
     case 16: e = launch_skinny<16>(st, 0, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;

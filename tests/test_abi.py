@@ -167,10 +167,12 @@ def test_linear_workspace_bytes(L):
     f = L.nvfp4_linear_workspace_bytes
     assert f(0, 64, 64) == 0 and f(8, 0, 64) == 0 and f(8, 64, 48) == 0
     m, n, k = 8, 1000, 2048
-    # quantized activations + partial maxima + (few tokens) split counters and 8 slabs
-    assert f(m, n, k) >= m * k // 2 + L.nvfp4_sf_bytes(m, k) + 16384 + 8 * m * n * 4
+    # quantized activations + partial maxima + (few tokens) counters and 9 slabs per tile
+    w_tiles = -(-n // 128)
+    slabs = w_tiles * 9 * m * 128 * 4
+    assert f(m, n, k) >= m * k // 2 + L.nvfp4_sf_bytes(m, k) + 16384 + slabs
     assert f(65, n, k) < f(64, n, k)         # no split workspace above 64 tokens
-    assert L.nvfp4_gemm_workspace_bytes(m, n, k) == 256 + 8 * m * n * 4
+    assert L.nvfp4_gemm_workspace_bytes(m, n, k) == 256 + slabs
     assert L.nvfp4_gemm_workspace_bytes(65, n, k) == 0
 
 
