@@ -165,7 +165,8 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k,
  * FP32 partial slabs: with fewer 128-row weight tiles than SMs, few-token
  * GEMMs deal the (tile, k-tile) iterations out to every SM in equal
  * contiguous shares (stream-K) and add the partial tiles in a fixed order;
- * else 0. Passing less (or NULL) is allowed and only disables the split. */
+ * else 0. Passing less (or NULL) is allowed and only disables the
+ * stream-K split. */
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -185,7 +186,7 @@ size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *   a_codes, b_codes: 16-byte aligned. a_sf, b_sf: 16-byte aligned.
  *   workspace  device scratch, nvfp4_gemm_workspace_bytes(m,n,k) bytes,
  *              16-byte aligned, or NULL; contents need no initialisation
- *              (the call zeroes the split counters itself).
+ *              (the call zeroes the reduction counters itself).
  * m <= 64 runs the few-token kernel (weights on the MMA's 128-row side,
  * tokens as its N); larger m the paired-CTA 256x256-tile kernel. Results do
  * not depend on the run: partial tiles are summed in k order.
@@ -202,7 +203,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
 
 /* Workspace bytes of nvfp4_linear: the quantized activations (codes, scales,
  * global), the amax pass's partial maxima and, for m <= 64, the few-token
- * GEMM's split counters and slabs. 0 for invalid sizes. */
+ * GEMM's reduction counters and slabs. 0 for invalid sizes. */
 size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*

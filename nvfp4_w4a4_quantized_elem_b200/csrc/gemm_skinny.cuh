@@ -2,7 +2,7 @@
 //
 // Same product as gemm_sm100.cuh (Y = dequant(A) dequant(B)^T / (g_a g_b)),
 // computed as Y^T = B A^T so that the weights fill the 128-row MMA side and
-// the tokens are the MMA N (16..256): the tensor cores then do no work on
+// the tokens are the MMA N (16, 32 or 64): the tensor cores then do no work on
 // padded token rows, and the kernel streams the weights at memory speed.
 // News article "Qwen3.8-27B最激进4bit量化开源，权重显存暴降2.9倍！" §02
 // (W4A4 on 4-bit tensor cores); decode throughput is one of the serving
@@ -71,7 +71,7 @@ enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, k
 
 template <int BNT>
 struct Cfg {
-  static_assert(BNT == 16 || BNT == 32 || BNT == 64 || BNT == 128 || BNT == 256, "token tile");
+  static_assert(BNT == 16 || BNT == 32 || BNT == 64, "token tile (few-token kernel: m <= 64)");
   static constexpr int A_BYTES = BW * BK_BYTES;             // 16 KiB of weights
   static constexpr int B_BYTES = (BNT < 8 ? 8 : BNT) * BK_BYTES;
   static constexpr int SFB_BLOCKS = (BNT + 127) / 128;      // 128-row scale blocks of tokens

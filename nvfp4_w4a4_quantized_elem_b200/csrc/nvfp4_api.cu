@@ -359,7 +359,7 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k, int6
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   (void)k;
   if (m < 1 || n < 1) return 0;
-  // few-token GEMMs split K across CTAs: split counters and FP32 slabs of Y
+  // few-token GEMMs share the work stream-K fashion: counters and FP32 slabs
   return m <= 64 ? skinny_workspace_bytes(m, n) : 0;
 }
 
@@ -433,9 +433,9 @@ nvfp4_status launch_skinny(DeviceState* st, int bit, const CUtensorMap& tmW, con
 }
 
 // Few tokens (m <= 64): Y^T = B A^T with the weights on the MMA's 128-row
-// side and the tokens as its N; K split across CTAs when the weight tiles
+// side and the tokens as its N; stream-K across all SMs when the weight tiles
 // cannot fill the GPU and a workspace (skinny_workspace_bytes) is given.
-// The split counters at the workspace's start are zeroed here when
+// The reduction counters at the workspace's start are zeroed here when
 // `zero_counters`, else the caller guarantees they are zero (every call
 // leaves them so). `early_w`: the weights were written before the previous
 // kernel in the stream started, so the kernel may read them before it ends.
@@ -446,7 +446,7 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                          void* workspace, size_t workspace_bytes, bool zero_counters,
                          int early_w, cudaStream_t s) {
   using namespace nvfp4::skinny;
-  const int bnt = m <= 16 ? 16 : m <= 32 ? 32 : m <= 64 ? 64 : m <= 128 ? 128 : 256;
+  const int bnt = m <= 16 ? 16 : m <= 32 ? 32 : 64;  // callers route m <= 64 here
   CUtensorMap tmW, tmX, tmSFW, tmSFX;
   if (nvfp4_status e = encode_2d(enc, &tmW, b_codes, static_cast<uint64_t>(k / 2),
                                  static_cast<uint64_t>(n), BW))
@@ -455,7 +455,7 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                                  static_cast<uint64_t>(m), static_cast<uint32_t>(bnt)))
     return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFW, b_sf, n, k, 1u)) return e;
-  if (nvfp4_status e = encode_sf(enc, &tmSFX, a_sf, m, k, bnt > 128 ? 2u : 1u)) return e;
+  if (nvfp4_status e = encode_sf(enc, &tmSFX, a_sf, m, k, 1u)) return e;
   Params p;
   p.M = static_cast<int>(m);
   p.N = static_cast<int>(n);
@@ -493,9 +493,7 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   switch (bnt) {
     case 16: e = launch_skinny<16>(st, 0, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
     case 32: e = launch_skinny<32>(st, 1, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
-    case 64: e = launch_skinny<64>(st, 2, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
-    case 128: e = launch_skinny<128>(st, 3, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
-    default: e = launch_skinny<256>(st, 4, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    default: e = launch_skinny<64>(st, 2, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
   }
   return e;
 }
@@ -618,7 +616,7 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (nvfp4_status e = get_encoder(&enc)) return e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // workspace: [split counters + slabs (m <= 64)][codes][scales][global][partials]
+  // workspace: [counters + slabs (m <= 64)][codes][scales][global][partials]
   uint8_t* w = static_cast<uint8_t*>(workspace);
   const size_t split_bytes = m <= 64 ? round_up(skinny_workspace_bytes(m, n), 256) : 0;
   uint8_t* a_codes = w + split_bytes;

@@ -197,7 +197,8 @@ def gemm(a: NVFP4Tensor, b: NVFP4Tensor, out: torch.Tensor | None = None,
          stream: torch.cuda.Stream | None = None) -> torch.Tensor:
     """nvfp4_gemm: Y[m, n] = dequant(A) @ dequant(B).T (A = activations
     [m, k], B = weights [n, k]); bf16 or fp32 output. ``workspace`` (at least
-    gemm_workspace_bytes) lets few-token GEMMs split K across the GPU."""
+    gemm_workspace_bytes) lets few-token GEMMs share the work across all SMs
+    (stream-K)."""
     if a.k != b.k:
         raise ValueError("k mismatch")
     m, n, k = a.rows, b.rows, a.k
