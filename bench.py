@@ -6,17 +6,22 @@
 A step is one pass of the hot path over one batch of seeded synthetic input:
 activation quantization (amax pass + quantizer, dynamic global scale) and the
 block-scaled FP4 GEMM against weights quantized beforehand (weights are
-offline in a W4A4 checkpoint). Workloads:
+offline in a W4A4 checkpoint); linear workloads run it as one nvfp4_linear
+call. Workloads:
   outlier    X 8192x5120 (8 channels x50) @ W 5120x5120        (default)
+  outlier_static  the same with a calibrated static activation global
   gdn_fused  X 8192x5120 @ fused qkv|z|a|b 12384x5120 (fold done offline)
   mlp32k     X 32768x5120 -> gate_up 34816 -> silu*mul -> requant -> down 5120
   mlp32k_fused  the same MLP with silu*mul + quantization of h fused into the
              gate_up GEMM epilogue (h's static global calibrated offline)
-  decode:M:K:N  few-token GEMM, e.g. decode:1:5120:17408 (HBM-bound)
+  decode:M:K:N  few-token layer, e.g. decode:1:5120:17408 (HBM-bound), replayed
+             as a CUDA graph
 Metric: TFLOP/s of the whole step (2*M*N*K per GEMM over quantize + GEMM
 time), with the GEMM's fraction of the dense FP4 tensor peak and the
 quantizer's GB/s alongside. Inputs stay resident in HBM; L2 (126 MB) is
-flushed by a 256 MiB write before every timed step, outside the timed events.
+flushed before every timed step, outside the timed events (256 MiB written,
+then 256 MiB read). The end-to-end figure moves X from and Y to pinned host
+memory every step (pipelined over three streams for prefill).
 
 Multi-GPU (torchrun): every rank runs the same step on its own batch (weak
 scaling, no collective on the data path); the per-rank device time is
@@ -45,7 +50,6 @@ sys.path.insert(0, ROOT)
 
 METRIC = "NVFP4 W4A4 GEMM TFLOPS incl. act quant, % dense FP4 peak; quant GB/s"
 FP4_SPEC_TFLOPS = 9000.0          # B200 dense FP4, public spec
-HBM_SPEC_GBS = 8000.0
 QUANT_BYTES_PER_ELEM = 2.5625     # read bf16 + write 0.5 code + 1/16 scale
 AMAX_BYTES_PER_ELEM = 2.0
 L2_FLUSH_BYTES = 256 << 20
