@@ -26,6 +26,11 @@
 //                    (Half a block per lane, the first layout, spent ~25% more
 //                    integer work per element; at 32768x17408 this layout
 //                    streams at 0.96 of the measured HBM bandwidth.)
+// L2 policy: the amax pass reads x with an evict-last hint, so that the
+// quantizer's second read of x is served from L2 as far as L2 holds it, and
+// the quantizer reads it with an evict-first hint, so that x's lines are the
+// first to leave L2 afterwards and the GEMM's operands stay (dynamic
+// quantization of 8192x5120: 39.9 -> 35.8 us; the bits are unchanged).
 // amax_b / 6 is computed as q = amax_b * RN(1/6), q + RN((amax_b - 6 q) *
 // RN(1/6)) with two FMAs; this equals the IEEE quotient for every
 // non-negative bf16 value (checked exhaustively with exact rationals in the
@@ -50,21 +55,37 @@ __device__ __forceinline__ float div6_rn(float a) {
   return __fmaf_rn(r, kInv6, q);
 }
 
-// 16-byte load through L1: the two halves of a lane's 32-byte block are
-// issued back to back and the second is served from the first's line fill.
-__device__ __forceinline__ uint4 ldg_l1(const void* p) {
+// L2 cache policies (createpolicy): every line the load touches gets the
+// policy's eviction priority.
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
+// 16-byte load through L1 with an L2 policy: the two halves of a lane's
+// 32-byte block are issued back to back and the second is served from the
+// first's line fill.
+__device__ __forceinline__ uint4 ldg_l1(const void* p, uint64_t pol) {
   uint4 v;
-  asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+               : "l"(p), "l"(pol));
   return v;
 }
 
-__device__ __forceinline__ uint4 ldg_stream(const void* p) {
+// 16-byte streaming load (no L1 allocation) with an L2 policy.
+__device__ __forceinline__ uint4 ldg_stream(const void* p, uint64_t pol) {
   uint4 v;
-  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+  asm volatile("ld.global.nc.L1::no_allocate.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-               : "l"(p));
+               : "l"(p), "l"(pol));
   return v;
 }
 
@@ -86,6 +107,7 @@ __global__ void __launch_bounds__(kAmaxThreads)
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const int64_t chunks = k >> 3;  // 16-byte chunks per row
   uint32_t m = 0;
+  const uint64_t pol = l2_evict_last_policy();  // the quantizer reads x next
   if (ldx == k) {
     // contiguous tensor: one flat stream of 16-byte chunks, 8 loads in flight
     const int64_t total = rows * chunks;
@@ -94,24 +116,24 @@ __global__ void __launch_bounds__(kAmaxThreads)
     for (; i + 7 * nthreads < total; i += 8 * nthreads) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = ldg_stream(x + (i + u * nthreads) * 8);
+      for (int u = 0; u < 8; ++u) v[u] = ldg_stream(x + (i + u * nthreads) * 8, pol);
 #pragma unroll
       for (int u = 0; u < 8; ++u) m = max(m, absmax_bits8(v[u]));
     }
-    for (; i < total; i += nthreads) m = max(m, absmax_bits8(ldg_stream(x + i * 8)));
+    for (; i < total; i += nthreads) m = max(m, absmax_bits8(ldg_stream(x + i * 8, pol)));
   }
   for (int64_t r = (ldx == k) ? rows : warp; r < rows; r += nwarps) {
     const uint16_t* row = x + r * ldx;
     int64_t c = lane;
     for (; c + 96 < chunks; c += 128) {
-      const uint4 v0 = ldg_stream(row + c * 8);
-      const uint4 v1 = ldg_stream(row + (c + 32) * 8);
-      const uint4 v2 = ldg_stream(row + (c + 64) * 8);
-      const uint4 v3 = ldg_stream(row + (c + 96) * 8);
+      const uint4 v0 = ldg_stream(row + c * 8, pol);
+      const uint4 v1 = ldg_stream(row + (c + 32) * 8, pol);
+      const uint4 v2 = ldg_stream(row + (c + 64) * 8, pol);
+      const uint4 v3 = ldg_stream(row + (c + 96) * 8, pol);
       m = max(m, max(max(absmax_bits8(v0), absmax_bits8(v1)),
                      max(absmax_bits8(v2), absmax_bits8(v3))));
     }
-    for (; c < chunks; c += 32) m = max(m, absmax_bits8(ldg_stream(row + c * 8)));
+    for (; c < chunks; c += 32) m = max(m, absmax_bits8(ldg_stream(row + c * 8, pol)));
   }
   m = __reduce_max_sync(0xFFFFFFFFu, m);
   __shared__ uint32_t s_red[32];
@@ -200,6 +222,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
   // of an atom's scales. Two passes cover the task's 4 atoms.
   const uint32_t jb = static_cast<uint32_t>(j & 3), ja = static_cast<uint32_t>(j >> 2);
   const uint32_t k32 = static_cast<uint32_t>(a.k);
+  const uint64_t pol = l2_evict_first_policy();  // x is not read again
   for (uint32_t t = w0; t < ntask; t += nw) {
     const uint32_t tl = t / nkc;
     const uint32_t kc = t - tl * nkc;
@@ -216,8 +239,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
       const uint32_t col = (kc * 4u + 2u * u + ja) * 64u + jb * 16u;
       v[u][0] = v[u][1] = make_uint4(0u, 0u, 0u, 0u);
       if (row_ok && col < k32) {
-        v[u][0] = ldg_l1(xrow + col);
-        v[u][1] = ldg_l1(xrow + col + 8);
+        v[u][0] = ldg_l1(xrow + col, pol);
+        v[u][1] = ldg_l1(xrow + col + 8, pol);
       }
     }
 #pragma unroll
