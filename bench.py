@@ -273,8 +273,9 @@ class Step:
             self.H = nvfp4.NVFP4Tensor.empty(m, ffn, dev)
             self.y = torch.empty((m, wk["n"]), dtype=torch.bfloat16, device=dev)
         self.launches = {"linear": 3, "mlp": 9, "mlp_fused": 4}[wk["kind"]]
-        if wk.get("x_global") is not None:
-            self.launches -= 1  # static global: no amax pass
+        one_pass = m * k * 2 <= nvfp4.ONE_PASS_MAX_BYTES  # quantizer takes the max itself
+        if wk.get("x_global") is not None or one_pass:
+            self.launches -= 1  # no amax pass
         if self.gws is not None:
             self.launches += 1  # split-counter clear of nvfp4_gemm
         self.graph = None
@@ -282,7 +283,8 @@ class Step:
         if self.fused_call:
             self.lws = nvfp4.linear_workspace(m, wk["W"].rows, k, dev)
         if wk.get("decode"):
-            self.launches = 3   # amax, quantizer, few-token GEMM (counters stay zero)
+            # [amax,] quantizer, few-token GEMM (the counters stay zero)
+            self.launches = 2 if one_pass else 3
             self.lws = nvfp4.linear_workspace(m, wk["W"].rows, k, dev)
             with torch.cuda.stream(stream):
                 nvfp4.linear(wk["x"], wk["W"], out=self.y, workspace=self.lws, stream=stream)
@@ -463,6 +465,7 @@ def run_gpu(args):
     stream.synchronize()
     qstatic_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in qev)
     amax_ms = max(q_avg_ms - qstatic_ms, 1e-6)
+    one_pass = m * k * 2 <= nvfp4.ONE_PASS_MAX_BYTES  # no separate amax pass to estimate
     elems = m * k
     quant_gbs = elems * QUANT_BYTES_PER_ELEM / (qstatic_ms * 1e-3) / 1e9
     amax_gbs = elems * AMAX_BYTES_PER_ELEM / (amax_ms * 1e-3) / 1e9
@@ -482,7 +485,9 @@ def run_gpu(args):
         step_gbs = step_bytes / (ms_per_step * 1e-3) / 1e9
         roofline = {"bound": "hbm", "achieved": round(step_gbs, 1), "peak": pk["hbm_gbs"],
                     "unit": "GB/s", "frac": round(step_gbs / pk["hbm_gbs"], 4), "traffic": traffic,
-                    "kernel": "nvfp4_linear step (amax + quantizer + skinny GEMM, overlapped)",
+                    "kernel": ("nvfp4_linear step (quantizer with the amax inside + skinny GEMM, "
+                               "overlapped)" if mm * kk * 2 <= nvfp4.ONE_PASS_MAX_BYTES else
+                               "nvfp4_linear step (amax + quantizer + skinny GEMM, overlapped)"),
                     "peak_source": f"measured copy bandwidth ({pk['source']})",
                     "algorithmic_bytes_per_launch": step_bytes}
     else:
@@ -516,10 +521,10 @@ def run_gpu(args):
         "components": {
             "phase_timing": phase_timing,
             "quantize_ms": round(q_avg_ms, 5), "gemm_ms": round(gemm_avg_ms, 5),
-            "quantizer_alone_ms": round(qstatic_ms, 5), "amax_ms_est": round(amax_ms, 5),
+            "quantizer_alone_ms": round(qstatic_ms, 5), "amax_ms_est": None if one_pass else round(amax_ms, 5),
             "quant_gbs": round(quant_gbs, 1),
             "quant_frac_hbm": round(quant_gbs / pk["hbm_gbs"], 4),
-            "amax_gbs": round(amax_gbs, 1),
+            "amax_gbs": None if one_pass else round(amax_gbs, 1),
             "hbm_peak_gbs": pk["hbm_gbs"],
             "quant_bytes_per_elem": QUANT_BYTES_PER_ELEM,
             "cublaslt_nvfp4_tflops": lib_ref,

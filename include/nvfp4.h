@@ -89,7 +89,9 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
  *   rows       >= 0 (0 writes nothing but global_out).
  *   k          > 0, k % 16 == 0.
  *   global_in  device FP32 scalar or NULL. NULL => dynamic mode: amax over x,
- *              g = 2688/amax (two kernels: an amax pass, then the quantizer).
+ *              g = 2688/amax (two kernels: an amax pass, then the quantizer;
+ *              one kernel when rows * k * 2 <= NVFP4_ONE_PASS_MAX_BYTES, in
+ *              which every CTA of the quantizer takes the max itself).
  *              Non-NULL => static (calibrated) mode: g = *global_in as given;
  *              block scales may then saturate at 448 and codes at +-6.
  *   codes      device, [rows][k/2] bytes, row pitch k/2; 4-byte aligned.
@@ -101,6 +103,7 @@ size_t nvfp4_quantize_workspace_bytes(int64_t rows, int64_t k);
  *              static mode). Contents need no initialisation.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED (k % 16), CUDA (launch).
  */
+#define NVFP4_ONE_PASS_MAX_BYTES 65536
 nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
                             const float* global_in, uint8_t* codes, uint8_t* sf,
                             float* global_out, void* workspace,

@@ -228,8 +228,9 @@ nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx
   const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
   if (n_tasks >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;  // 32-bit task index
   if (nvfp4_status e = quant_occupancy(st)) return e;
-  int nparts = 0;
-  if (global_in == nullptr) {
+  static_assert(kSelfAmaxBytes == NVFP4_ONE_PASS_MAX_BYTES, "one-pass bound of nvfp4.h");
+  int nparts = 0;  // dynamic mode with nparts == 0: the quantizer takes the max itself
+  if (global_in == nullptr && rows * k * 2 > kSelfAmaxBytes) {
     const int64_t blocks = amax_blocks(rows, k, ldx, st);
     if (blocks > max_parts) return NVFP4_ERR_UNSUPPORTED;
     nparts = static_cast<int>(blocks);

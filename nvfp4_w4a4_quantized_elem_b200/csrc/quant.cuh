@@ -46,6 +46,7 @@ constexpr int kAmaxThreads = 1024;
 constexpr int kMaxPartials = 4096;            // workspace = 16 KiB
 constexpr int kQuantThreads = 256;
 constexpr int kAtomsPerTask = 4;
+constexpr int64_t kSelfAmaxBytes = 64 * 1024;  // x up to this size: no amax pass
 constexpr float kInv6 = 0.16666667163372039794921875f;  // RN(1/6) = 0x3E2AAAAB
 
 // RN(a / 6) for a non-negative bf16 value a (see the header comment).
@@ -151,7 +152,7 @@ struct QuantArgs {
   int64_t rows, k, ldx;
   const float* global_in;   // static mode when non-null
   const float* partials;    // dynamic mode: per-CTA maxima of amax_kernel
-  int nparts;
+  int nparts;               // dynamic mode: 0 = no amax pass, every CTA reads x itself
   uint8_t* codes;
   uint8_t* sf;
   float* global_out;
@@ -174,8 +175,33 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
     if (threadIdx.x == 0) s_g = *a.global_in;
   } else {
     uint32_t m = 0;
-    for (int i = threadIdx.x; i < a.nparts; i += blockDim.x)
-      m = max(m, __float_as_uint(a.partials[i]));  // non-negative: bits order as values
+    if (a.nparts > 0) {
+      for (int i = threadIdx.x; i < a.nparts; i += blockDim.x)
+        m = max(m, __float_as_uint(a.partials[i]));  // non-negative: bits order as values
+    } else {
+      // small x (the host bounds it by kSelfAmaxBytes): every CTA takes the
+      // tensor's max itself from L2, so no amax pass precedes this kernel
+      // (8 loads in flight per thread: x of one 17408-wide row is 2176
+      // chunks, which one dependent load per round would take 9 round trips)
+      const uint32_t chunks = static_cast<uint32_t>(a.k >> 3);
+      const uint32_t total = static_cast<uint32_t>(a.rows) * chunks;
+      const uint32_t nt = blockDim.x;
+      auto chunk = [&](uint32_t i) {
+        const uint32_t r = i / chunks;
+        const uint32_t c = i - r * chunks;
+        return __ldg(reinterpret_cast<const uint4*>(
+            a.x + static_cast<uint64_t>(r) * static_cast<uint64_t>(a.ldx) + c * 8u));
+      };
+      uint32_t i = threadIdx.x;
+      for (; i + 7u * nt < total; i += 8u * nt) {
+        uint4 v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v[u] = chunk(i + u * nt);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m = max(m, absmax_bits8(v[u]) << 16);  // -> FP32 bits
+      }
+      for (; i < total; i += nt) m = max(m, absmax_bits8(chunk(i)) << 16);
+    }
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     if (lane == 0) s_red[wib] = m;
     __syncthreads();

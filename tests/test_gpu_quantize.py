@@ -119,3 +119,28 @@ def test_quantize_deterministic_and_reuses_workspace(nv, orc):
     b = nv.quantize(x, workspace=ws)
     assert torch.equal(a.codes, b.codes) and torch.equal(a.sf, b.sf)
     assert torch.equal(a.global_scale, b.global_scale)
+
+
+@pytest.mark.parametrize("rows,k", [(2, 16384), (2, 16400), (1, 32768), (3, 16384)])
+def test_quantize_one_pass_bound(nv, orc, rows, k):
+    """Dynamic quantization on both sides of NVFP4_ONE_PASS_MAX_BYTES (64 KiB
+    of x: one kernel that takes the max itself; above it: amax pass, then
+    the quantizer). The tensor's largest magnitude sits in the last element,
+    so a max that stops short of the end changes g and every scale."""
+    x = gaussian(rows, k, seed=rows + k)
+    x[-1, -1] = -40.0
+    assert (rows * k * 2 <= nv.ONE_PASS_MAX_BYTES) == (rows * k <= 32768)
+    out, ref = check(nv, orc, x, what=f"{rows}x{k}")
+    assert out.global_scale.item() == np.float32(2688.0) / np.float32(40.0)
+
+
+@pytest.mark.parametrize("rows", [70, 300])
+def test_quantize_dynamic_ignores_row_padding(nv, orc, rows):
+    """x with ldx > k and a large value in every row's padding: the global
+    comes from the first k columns only, in the one-kernel path (70 rows,
+    22 KiB) and behind the amax pass (300 rows, 94 KiB)."""
+    base = gaussian(rows, 256, seed=rows)
+    base[:, 160:] = 1.0e4
+    out = nv.quantize(base.cuda()[:, :160])
+    ref = orc.quantize(bits(base[:, :160].contiguous()))
+    assert_quant_equal(out, ref, f"padded rows={rows}")
