@@ -181,26 +181,27 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
     } else {
       // small x (the host bounds it by kSelfAmaxBytes): every CTA takes the
       // tensor's max itself from L2, so no amax pass precedes this kernel
-      // (8 loads in flight per thread: x of one 17408-wide row is 2176
-      // chunks, which one dependent load per round would take 9 round trips)
+      // Rounds of 8 predicated 16-byte loads per thread, all in flight
+      // before the first max: x of at most 64 KiB takes 2 round trips
+      // (one dependent load at a time took 9 for a 17408-wide row).
       const uint32_t chunks = static_cast<uint32_t>(a.k >> 3);
       const uint32_t total = static_cast<uint32_t>(a.rows) * chunks;
       const uint32_t nt = blockDim.x;
-      auto chunk = [&](uint32_t i) {
-        const uint32_t r = i / chunks;
-        const uint32_t c = i - r * chunks;
-        return __ldg(reinterpret_cast<const uint4*>(
-            a.x + static_cast<uint64_t>(r) * static_cast<uint64_t>(a.ldx) + c * 8u));
-      };
-      uint32_t i = threadIdx.x;
-      for (; i + 7u * nt < total; i += 8u * nt) {
+      for (uint32_t i = threadIdx.x; i < total; i += 8u * nt) {
         uint4 v[8];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) v[u] = chunk(i + u * nt);
+        for (int u = 0; u < 8; ++u) {
+          const uint32_t e = i + u * nt;
+          const uint32_t r = e / chunks;
+          const uint32_t c = e - r * chunks;
+          v[u] = e < total ? __ldg(reinterpret_cast<const uint4*>(
+                                 a.x + static_cast<uint64_t>(r) * static_cast<uint64_t>(a.ldx) +
+                                 c * 8u))
+                           : make_uint4(0u, 0u, 0u, 0u);
+        }
 #pragma unroll
         for (int u = 0; u < 8; ++u) m = max(m, absmax_bits8(v[u]) << 16);  // -> FP32 bits
       }
-      for (; i < total; i += nt) m = max(m, absmax_bits8(chunk(i)) << 16);
     }
     m = __reduce_max_sync(0xFFFFFFFFu, m);
     if (lane == 0) s_red[wib] = m;
