@@ -4,7 +4,8 @@
                     [--impl reference]
 
 A step is one pass of the hot path over one batch of seeded synthetic input:
-activation quantization (amax pass + quantizer, dynamic global scale) and the
+activation quantization (amax pass + quantizer, dynamic global scale; the
+quantizer alone takes the max of a decode step's few tokens) and the
 block-scaled FP4 GEMM against weights quantized beforehand (weights are
 offline in a W4A4 checkpoint); linear workloads run it as one nvfp4_linear
 call. Workloads:
@@ -339,15 +340,41 @@ class Step:
         return y
 
 
-def kernel_source_hash() -> str:
-    """Hash of every kernel source: a DRAM-traffic figure is only reported
-    while the kernels are the ones it was measured on."""
-    d = os.path.join(ROOT, "nvfp4_w4a4_quantized_elem_b200", "csrc")
+def code_tokens(src: str) -> str:
+    """C/CUDA source without its comments, whitespace runs collapsed: what
+    the compiler sees of it (string and character literals kept whole)."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_source_hash(csrc: str | None = None) -> str:
+    """Hash of the code of every kernel source (comments and layout
+    excluded): a DRAM-traffic figure is only reported while the kernels are
+    the ones it was measured on."""
+    d = csrc or os.path.join(ROOT, "nvfp4_w4a4_quantized_elem_b200", "csrc")
     h = hashlib.sha256()
     for f in sorted(os.listdir(d)):
         if f.endswith((".cu", ".cuh")):
             h.update(f.encode())
-            h.update(open(os.path.join(d, f), "rb").read())
+            h.update(code_tokens(open(os.path.join(d, f), encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -219,8 +219,9 @@ size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * relies on W, w_sf and w_global being written before the call (by work
  * already in the stream or earlier), never by a kernel launched in between.
  *   x         device bf16 [m][ldx], 16-byte aligned, ldx >= k, ldx % 8 == 0.
- *   x_global  NULL: dynamic global scale of X (amax pass); else a device FP32
- *             static global (e.g. from nvfp4_calibrate_global).
+ *   x_global  NULL: dynamic global scale of X (amax pass, or none for X of at
+ *             most NVFP4_ONE_PASS_MAX_BYTES, as in nvfp4_quantize); else a
+ *             device FP32 static global (e.g. from nvfp4_calibrate_global).
  *   w_codes, w_sf, w_global  weights [n][k] in NVFP4 (as nvfp4_gemm's B).
  *   y, y_dtype, ldy          as nvfp4_gemm.
  *   m, n >= 1; k % 32 == 0.

@@ -218,8 +218,9 @@ nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
 }
 
 // Dynamic or static NVFP4 quantization of x (arguments already checked):
-// the amax pass (dynamic only) into `partials` (at most max_parts CTAs),
-// then the quantizer, launched to overlap the amax pass's tail.
+// the amax pass (dynamic only, x above kSelfAmaxBytes) into `partials` (at
+// most max_parts CTAs), then the quantizer, launched to overlap the amax
+// pass's tail; dynamic x up to kSelfAmaxBytes: the quantizer alone.
 nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx,
                              const float* global_in, uint8_t* codes, uint8_t* sf,
                              float* global_out, float* partials, int64_t max_parts,

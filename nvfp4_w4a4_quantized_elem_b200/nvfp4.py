@@ -131,7 +131,8 @@ def quantize(x: torch.Tensor, global_scale: torch.Tensor | None = None,
              out: NVFP4Tensor | None = None, workspace: torch.Tensor | None = None,
              stream: torch.cuda.Stream | None = None) -> NVFP4Tensor:
     """nvfp4_quantize: bf16 [rows, k] (rows may be strided) -> NVFP4Tensor.
-    ``global_scale`` None => dynamic global (amax pass + quantizer)."""
+    ``global_scale`` None => dynamic global (amax pass + quantizer; one
+    kernel when x is at most ONE_PASS_MAX_BYTES)."""
     _require_cuda(x, "x", torch.bfloat16)
     if x.dim() != 2 or x.stride(1) != 1:
         raise ValueError("x must be 2-D with unit stride along k")
