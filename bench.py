@@ -466,6 +466,8 @@ def run_gpu(args):
         quant_ms, gemm_ms = separate_phases(step, wk, stream, flush)
         phase_timing = ("quantizer and GEMM each launched alone after the timed steps, "
                         "20 times, CUDA events on their stream, L2 flushed before each")
+    cpu_leg = rank == 0 and world == 1 and not args.no_cpu_baseline
+    gpu_sample = sample_outputs(step) if cpu_leg and wk["kind"] == "linear" else None
     total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / args.steps
     value = job_throughput(flops, world, ms_per_step)
@@ -563,8 +565,9 @@ def run_gpu(args):
         "gpu_launches": step.launches * args.steps,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(oracle_name(args.workload), budget_s=args.cpu_seconds)
+    if cpu_leg:
+        out["cpu_baseline"] = cpu_baseline(oracle_name(args.workload), budget_s=args.cpu_seconds,
+                                           gpu_sample=gpu_sample, workload=args.workload)
     if rank == 0:
         print(json.dumps(out), flush=True)
     if dist is not None:
@@ -783,7 +786,7 @@ def cpu_model() -> str:
     return "unknown"
 
 
-def cpu_baseline(name, budget_s=15.0, rows=128):
+def cpu_baseline(name, budget_s=15.0, rows=128, gpu_sample=None, workload=None):
     orc, w = oracle_workload(name)
     rows = min(rows, len(w["x_bits"]))
     oracle_sample_step(orc, w, 8)  # warm (builds/loads the oracle)
@@ -805,7 +808,71 @@ def cpu_baseline(name, budget_s=15.0, rows=128):
         k = w["x_bits"].shape[1]
         out["quant_gbs"] = round(reps * rows * k * QUANT_BYTES_PER_ELEM / times["quant"] / 1e9, 4)
         out["gemm_gflops"] = round(w["flops_per_row"] * rows * reps / times["gemm"] / 1e9, 2)
+    if gpu_sample is not None:
+        try:
+            out["parity"] = oracle_parity(orc, w, workload or name, gpu_sample)
+        except Exception as e:  # a report field: never lose the measured line over it
+            out["parity"] = {"pass": False, "error": f"{type(e).__name__}: {e}"}
     return out
+
+
+def sample_outputs(step, rows=128):
+    """The first rows of the measured step's Y and of its quantized X (codes,
+    the first 128-row block of swizzled scales, global), copied to the host
+    for the oracle leg. Taken right after the timed steps and the phase
+    timing, whose launches all compute these same values."""
+    r = min(rows, step.y.shape[0])
+    block = 128 * (-(-step.A.k // 64) * 4)  # one row block of swizzled scales
+    if step.y.is_cuda:
+        torch.cuda.synchronize()
+    return dict(rows=r, y=step.y[:r].float().cpu().numpy(),
+                codes=step.A.codes[:r].cpu().numpy(), sf=step.A.sf[:block].cpu().numpy(),
+                g=step.A.global_scale.cpu().numpy()[0])
+
+
+def oracle_parity(orc, w, workload, gpu):
+    """The measured step against the oracle on its first rows: the oracle
+    takes the activation global the step uses from the seeded inputs itself
+    (2688 / amax over the whole X; for outlier_static the running amax over
+    the four calibration batches), quantizes those rows with it, and must
+    match the GPU's codes, scales and global bit for bit; Y must lie within
+    the GEMM tolerance (relative Frobenius <= 1e-3 against the FP64 result
+    rounded to bf16, and per element <= 2e-2 * ||x_hat_m|| * ||w_hat_n||)."""
+    import numpy as np
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+
+    def bits(t):
+        return t.contiguous().view(torch.int16).numpy().view(np.uint16)
+
+    if workload == "outlier_static":
+        cfg = wl.outlier()
+        amax = np.float32(0.0)
+        for seed in (101, 102, 103, 104):
+            cfg.x_seed = seed
+            amax = max(amax, orc.tensor_amax(bits(cfg.x())))
+    elif workload == "outlier":
+        amax = orc.tensor_amax(bits(wl.outlier().x()))
+    elif workload == "gdn_fused":
+        amax = orc.tensor_amax(bits(wl.gdn_fused().x()))
+    else:  # decode: the sample is the whole X
+        amax = orc.tensor_amax(w["x_bits"])
+    g = orc.global_from_amax(amax)
+    r = gpu["rows"]
+    qa = orc.quantize(np.ascontiguousarray(w["x_bits"][:r]), global_in=g)
+    x_exact = (np.array_equal(gpu["codes"], qa.codes) and np.array_equal(gpu["sf"], qa.sf_swizzled)
+               and np.float32(gpu["g"]).view(np.uint32) == np.float32(g).view(np.uint32))
+    ref = torch.from_numpy(orc.gemm(qa, w["qw"])).to(torch.bfloat16).double().numpy()
+    err = gpu["y"].astype(np.float64) - ref
+    fro = float(np.linalg.norm(err) / max(np.linalg.norm(ref), 1e-300))
+    qw = w["qw"]
+    col = np.concatenate([np.linalg.norm(orc.dequantize_rows(qw, np.arange(i, min(i + 1024, qw.rows))),
+                                         axis=1) for i in range(0, qw.rows, 1024)])
+    row = np.linalg.norm(orc.dequantize(qa), axis=1)
+    excess = float(np.max(np.abs(err) - 2e-2 * row[:, None] * col[None, :]))
+    ok = bool(x_exact and fro <= 1e-3 and excess <= 0.0 and np.all(np.isfinite(gpu["y"])))
+    return {"rows": r, "x_codes_scales_global_bit_exact": bool(x_exact),
+            "y_rel_fro": fro, "y_rel_fro_limit": 1e-3,
+            "y_worst_excess_over_elem_bound": excess, "pass": ok}
 
 
 def run_reference(args):

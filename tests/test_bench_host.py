@@ -45,3 +45,38 @@ def test_traffic_is_reported_only_for_the_measured_kernels():
         got = bench.dram_traffic(name)
         assert got == (float(e["dram_bytes_per_launch"]) if e["csrc_sha256_16"] == now else None)
     assert bench.dram_traffic("no such workload") is None
+
+
+def test_oracle_parity_leg_accepts_the_oracle_and_flags_a_planted_error():
+    """The bench's parity report on the oracle's own outputs passes; a flipped
+    code byte or a Y element off by far more than the tolerance fails it
+    (the plant is made in the oracle's copy, on the CPU)."""
+    import types
+
+    import numpy as np
+    import torch
+
+    import oracle as orc
+    name = "decode:3:256:384"
+    o, w = bench.oracle_workload(name)
+    amax = o.tensor_amax(w["x_bits"])
+    qa = o.quantize(np.ascontiguousarray(w["x_bits"]), global_in=o.global_from_amax(amax))
+    y = torch.from_numpy(o.gemm(qa, w["qw"])).to(torch.bfloat16)
+    A = types.SimpleNamespace(codes=torch.from_numpy(qa.codes.copy()),
+                              sf=torch.from_numpy(qa.sf_swizzled.copy()),
+                              global_scale=torch.tensor([float(qa.g)], dtype=torch.float32), k=256)
+    step = types.SimpleNamespace(y=y, A=A)
+    good = bench.sample_outputs(step)
+    rep = bench.oracle_parity(orc, w, name, good)
+    assert rep["pass"] and rep["x_codes_scales_global_bit_exact"] and rep["rows"] == 3
+    assert rep["y_rel_fro"] == 0.0
+
+    bad = dict(good, codes=good["codes"].copy())
+    bad["codes"][1, 7] ^= 0x01
+    rep = bench.oracle_parity(orc, w, name, bad)
+    assert not rep["pass"] and not rep["x_codes_scales_global_bit_exact"]
+
+    bad = dict(good, y=good["y"].copy())
+    bad["y"][2, 5] += 1.0e3
+    rep = bench.oracle_parity(orc, w, name, bad)
+    assert not rep["pass"] and rep["y_worst_excess_over_elem_bound"] > 0
