@@ -550,7 +550,8 @@ def run_gpu(args):
         "components": {
             "phase_timing": phase_timing,
             "quantize_ms": round(q_avg_ms, 5), "gemm_ms": round(gemm_avg_ms, 5),
-            "quantizer_alone_ms": round(qstatic_ms, 5), "amax_ms_est": None if one_pass else round(amax_ms, 5),
+            "quantizer_alone_ms": round(qstatic_ms, 5),
+            "amax_ms_est": None if one_pass else round(amax_ms, 5),
             "quant_gbs": round(quant_gbs, 1),
             "quant_frac_hbm": round(quant_gbs / pk["hbm_gbs"], 4),
             "amax_gbs": None if one_pass else round(amax_gbs, 1),
