@@ -32,6 +32,14 @@ def test_header_declares_the_boundary():
         assert f in names
 
 
+def test_binding_constants_match_the_header():
+    """Constants the binding mirrors from include/nvfp4.h."""
+    from nvfp4_w4a4_quantized_elem_b200 import nvfp4
+    text = open(HEADER).read()
+    m = re.search(r"#define NVFP4_ONE_PASS_MAX_BYTES (\d+)", text)
+    assert m and int(m.group(1)) == nvfp4.ONE_PASS_MAX_BYTES
+
+
 def test_library_exports_every_declared_symbol(L):
     from nvfp4_w4a4_quantized_elem_b200 import nvfp4
     names = declared_functions()
