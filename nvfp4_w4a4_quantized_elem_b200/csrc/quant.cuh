@@ -179,11 +179,11 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
       for (int i = threadIdx.x; i < a.nparts; i += blockDim.x)
         m = max(m, __float_as_uint(a.partials[i]));  // non-negative: bits order as values
     } else {
-      // small x (the host bounds it by kSelfAmaxBytes): every CTA takes the
-      // tensor's max itself from L2, so no amax pass precedes this kernel
+      // Small x (the host bounds it by kSelfAmaxBytes): every CTA takes the
+      // tensor's max itself from L2, so no amax pass precedes this kernel.
       // Rounds of 8 predicated 16-byte loads per thread, all in flight
-      // before the first max: x of at most 64 KiB takes 2 round trips
-      // (one dependent load at a time took 9 for a 17408-wide row).
+      // before the first max: x of at most 64 KiB takes 2 round trips (one
+      // dependent load at a time took 9 for a 17408-wide row).
       const uint32_t chunks = static_cast<uint32_t>(a.k >> 3);
       const uint32_t total = static_cast<uint32_t>(a.rows) * chunks;
       const uint32_t nt = blockDim.x;
