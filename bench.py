@@ -123,12 +123,17 @@ class ClockSampler:
         if self.thread is not None:
             self.thread.join(timeout=2)
 
-    def summary(self, t0: float, t1: float):
+    def summary(self, t0: float, t1: float, extended: bool = False):
+        """Median SM clock, max clock and the throttle reasons seen between t0
+        and t1: the timed region, or (`extended`) the timed region followed by
+        a second of the same step when the timed region alone is shorter than
+        a few sample periods. Fewer than 3 samples there: the whole run."""
         rows = [s for (t, s) in self.samples if t0 <= t <= t1]
-        window = "timed region"
-        if len(rows) < 3:  # timed region shorter than a few sample periods
+        window = ("timed region + 1 s of the same step (timed region shorter than the "
+                  "sample period)" if extended else "timed region")
+        if len(rows) < 3:
             rows = [s for (_, s) in self.samples]
-            window = "whole run (timed region shorter than 3 samples)"
+            window = "whole run (fewer than 3 samples in the timed window)"
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for r in rows:
@@ -446,6 +451,7 @@ def run_gpu(args):
         dist.barrier()
     # one extra second of the same step for the clock record if the timed
     # region was shorter than a few sample periods (not part of any number)
+    t2 = t1
     if t1 - t0 < 1.0:
         with torch.cuda.stream(stream):
             end = time.time() + 1.0
@@ -453,8 +459,9 @@ def run_gpu(args):
                 for _ in range(20):
                     step.run()
                 stream.synchronize()
+        t2 = time.time()
     sampler.stop()
-    clocks = sampler.summary(t0, t1)
+    clocks = sampler.summary(t0, t2, extended=t2 > t1)
 
     step_ms = [events[i][0].elapsed_time(events[i][nph - 1]) for i in range(args.steps)]
     if not step.fused_call:

@@ -80,3 +80,25 @@ def test_oracle_parity_leg_accepts_the_oracle_and_flags_a_planted_error():
     bad["y"][2, 5] += 1.0e3
     rep = bench.oracle_parity(orc, w, name, bad)
     assert not rep["pass"] and rep["y_worst_excess_over_elem_bound"] > 0
+
+
+def test_clock_summary_window_and_reasons():
+    """The clock record: median SM clock and the throttle reasons seen in the
+    timed window (extended by the extra second of the same step), idle
+    samples outside it ignored; too few samples fall back to the whole run."""
+    s = bench.ClockSampler(0)
+
+    def row(mhz, power_cap="Not Active", thermal="Not Active"):
+        return f"0, {mhz}, 1965, 900.0, 0x4, Not Active, Not Active, {thermal}, {power_cap}"
+
+    s.samples = [(0.0, row(345)), (0.5, row(345))]                  # idle before the run
+    s.samples += [(1.0 + 0.1 * i, row(1700 + i, power_cap="Active")) for i in range(10)]
+    s.samples += [(5.0, row(300, thermal="Active"))]                 # idle after the run
+    c = s.summary(1.0, 2.0, extended=True)
+    assert c["samples"] == 10 and c["sm_mhz"] == 1704.5 and c["sm_max_mhz"] == 1965.0
+    assert c["reasons"] == ["sw_power_cap"] and c["window"].startswith("timed region + 1 s")
+    c = s.summary(1.0, 1.15)                                         # 2 samples: whole run
+    assert c["samples"] == 13 and c["window"].startswith("whole run")
+    assert c["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
+    s.samples = [(1.0, "garbage"), (1.1, "0, N/A, N/A")]
+    assert s.summary(0.0, 2.0) is None
