@@ -87,7 +87,7 @@ def peaks():
 
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled every 100 ms."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -111,7 +111,21 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.samples.append((time.time(), line.strip()))
+            self.samples.append(self.parse(line, time.time()))
+
+    @staticmethod
+    def parse(line: str, arrival: float):
+        """(sample time, fields after the timestamp). The time is nvidia-smi's
+        own stamp (local time, "YYYY/MM/DD HH:MM:SS.mmm"), so output that a
+        pipe delivers in bursts still lands in the right window; the arrival
+        time if the stamp does not parse (the field is dropped either way)."""
+        stamp, _, rest = line.strip().partition(",")
+        try:
+            whole, _, ms = stamp.strip().partition(".")
+            t = time.mktime(time.strptime(whole, "%Y/%m/%d %H:%M:%S")) + float("0." + (ms or "0"))
+        except ValueError:
+            t = arrival
+        return t, rest.strip()
 
     def stop(self):
         if self.proc is not None:

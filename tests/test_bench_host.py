@@ -102,3 +102,12 @@ def test_clock_summary_window_and_reasons():
     assert c["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
     s.samples = [(1.0, "garbage"), (1.1, "0, N/A, N/A")]
     assert s.summary(0.0, 2.0) is None
+
+
+def test_clock_sample_uses_nvidia_smi_timestamp():
+    import time
+    line = "2026/12/02 21:25:18.250, 0, 1700, 1965, 900.0, 0x4, Not Active, Not Active, Not Active, Active\n"
+    t, rest = bench.ClockSampler.parse(line, arrival=123.0)
+    assert abs(t - (time.mktime(time.strptime("2026/12/02 21:25:18", "%Y/%m/%d %H:%M:%S")) + 0.25)) < 1e-6
+    assert rest.startswith("0, 1700, 1965")
+    assert bench.ClockSampler.parse("no stamp, 0, 1700", arrival=123.0) == (123.0, "0, 1700")
