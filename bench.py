@@ -96,13 +96,21 @@ class ClockSampler:
         self.samples = []
         self.proc = None
         self.thread = None
+        self.stamped = True
+
+    def _spawn(self, query: str):
+        return subprocess.Popen(
+            ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={query}",
+             "--format=csv,noheader,nounits", "-lms", "100"],
+            stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = self._spawn(self.Q)
+            time.sleep(0.3)
+            if self.proc.poll() is not None:  # query refused: sample without the stamp
+                self.stamped = False
+                self.proc = self._spawn(self.Q.partition(",")[2])
         except Exception:
             self.proc = None
             return
@@ -111,7 +119,8 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.samples.append(self.parse(line, time.time()))
+            now = time.time()
+            self.samples.append(self.parse(line, now) if self.stamped else (now, line.strip()))
 
     @staticmethod
     def parse(line: str, arrival: float):
