@@ -121,6 +121,16 @@ class ClockSampler:
         for line in self.proc.stdout:
             now = time.time()
             self.samples.append(self.parse(line, now) if self.stamped else (now, line.strip()))
+        # the stamped query was refused after the start-up check: sample
+        # again without the stamp (arrival times) for the rest of the run
+        if self.stamped and not self.samples and self.proc.poll() not in (None, 0):
+            self.stamped = False
+            try:
+                self.proc = self._spawn(self.Q.partition(",")[2])
+            except Exception:
+                return
+            for line in self.proc.stdout:
+                self.samples.append((time.time(), line.strip()))
 
     @staticmethod
     def parse(line: str, arrival: float):
@@ -172,7 +182,13 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(name)
         if not sm:
-            return None
+            # say why there is no clock record instead of a bare null
+            rc = None if self.proc is None else self.proc.poll()
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "window": window,
+                    "error": ("nvidia-smi could not be started" if self.proc is None else
+                              f"nvidia-smi gave no parseable samples (exit code {rc}, "
+                              f"{'stamped' if self.stamped else 'unstamped'} query)")}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
                 "samples": len(sm), "window": window}
 

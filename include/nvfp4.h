@@ -124,12 +124,17 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
  * Arguments, layouts, results and errors are those of nvfp4_quantize (minus
  * the workspace pair). Additionally:
  *   - NVFP4_ERR_UNSUPPORTED if the amax pass would need more than
- *     NVFP4_NOALLOC_MAX_PARTIALS CTAs (it launches at most 2 x SM count of
- *     them; 296 on a 148-SM B200).
- *   - The first call on a device looks up the array's device address
+ *     NVFP4_NOALLOC_MAX_PARTIALS CTAs. Its grid is capped at one resident
+ *     wave (SM count x resident amax CTAs per SM, from an occupancy query):
+ *     296 on a 148-SM B200 today; the cap is checked on every call, so a
+ *     device or build with a larger wave gets this error, never an overrun.
+ *   - The first call in a CUDA context looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
- *     before any stream capture. Later calls allocate nothing and call no
- *     allocating routine.
+ *     before any stream capture. The library keys the address on the
+ *     context's unique id, so after a device reset (which reloads the module,
+ *     possibly at another address) the next call looks it up again; that
+ *     call, too, should come before any capture. Other calls allocate
+ *     nothing and call no allocating routine.
  *   - Every call on a device shares the one array and it keeps the last
  *     call's contents. Nothing in it needs to start at zero: each slot the
  *     quantizer reads is first written by the same call's amax pass. Calls

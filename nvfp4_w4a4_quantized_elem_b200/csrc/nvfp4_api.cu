@@ -29,28 +29,83 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 
+// What the library caches per device. Everything here belongs to one CUDA
+// context: function attributes, occupancy and symbol addresses are properties
+// of the module loaded into that context, and a device reset (or any other
+// teardown of the primary context) loads the module again, possibly at other
+// addresses. The state is therefore keyed on the context's process-unique id
+// (cuCtxGetId) and rebuilt when the current context changes. One context per
+// device at a time is assumed (the runtime's primary context, as torch and
+// most callers use); threads that drive two contexts of one device at once
+// would rebuild each other's state.
 struct DeviceState {
+  unsigned long long ctx_id = 0;      // context the fields below belong to (0 = none yet)
   int sms = 0;
   bool gemm_smem_set = false;
   unsigned skinny_smem_set = 0;       // bit per token-tile instantiation
   int amax_per_sm = 0;                // resident CTAs per SM of the quantizer's kernels
   int quant_per_sm = 0;
-  float* noalloc_partials = nullptr;  // device address of g_noalloc_partials
+  float* noalloc_partials = nullptr;  // device address of g_noalloc_partials in ctx_id
 };
 
 std::mutex g_mutex;
 DeviceState g_dev[kMaxDevices];
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+PFN_cuCtxGetCurrent_v4000 g_ctx_current = nullptr;
+PFN_cuCtxGetId_v12000 g_ctx_id = nullptr;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+nvfp4_status driver_entry(const char* name, int version, void** fn) {
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion(name, fn, version, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || *fn == nullptr) {
+    cudaGetLastError();
+    return NVFP4_ERR_CUDA;
+  }
+  return NVFP4_OK;
+}
+
+// Unique id of the context current on this thread for device `dev`; binds
+// the device's primary context first if the runtime has not done so yet on
+// this thread (cudaSetDevice initialises it; the device stays the same).
+nvfp4_status current_context_id(int dev, unsigned long long* id) {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* a = nullptr;
+    void* b = nullptr;
+    if (driver_entry("cuCtxGetCurrent", 4000, &a) == NVFP4_OK &&
+        driver_entry("cuCtxGetId", 12000, &b) == NVFP4_OK) {
+      g_ctx_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(a);
+      g_ctx_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(b);
+    }
+  });
+  if (g_ctx_current == nullptr || g_ctx_id == nullptr) return NVFP4_ERR_CUDA;
+  CUcontext ctx = nullptr;
+  if (g_ctx_current(&ctx) != CUDA_SUCCESS) return NVFP4_ERR_CUDA;
+  if (ctx == nullptr) {
+    if (cudaSetDevice(dev) != cudaSuccess) {
+      cudaGetLastError();
+      return NVFP4_ERR_CUDA;
+    }
+    if (g_ctx_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return NVFP4_ERR_CUDA;
+  }
+  return g_ctx_id(ctx, id) == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
+}
 
 nvfp4_status current_device(int* dev, DeviceState** st) {
   if (cudaGetDevice(dev) != cudaSuccess || *dev < 0 || *dev >= kMaxDevices) {
     cudaGetLastError();
     return NVFP4_ERR_CUDA;
   }
+  unsigned long long id = 0;
+  if (nvfp4_status e = current_context_id(*dev, &id)) return e;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceState& s = g_dev[*dev];
+  if (s.ctx_id != id) {  // first call in this context: nothing cached applies
+    s = DeviceState{};
+    s.ctx_id = id;
+  }
   if (s.sms == 0) {
     int sms = 0;
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, *dev) != cudaSuccess ||
@@ -199,10 +254,12 @@ int64_t amax_blocks(int64_t rows, int64_t k, int64_t ldx, const DeviceState* st)
 
 // Scratch of nvfp4_quantize_noalloc: the amax pass's per-CTA partial maxima.
 // Host code must not use this name as a pointer (it is a host-side stand-in);
-// the device address comes from cudaGetSymbolAddress, once per device.
+// the device address comes from cudaGetSymbolAddress, once per device and
+// context (current_device() clears the cached address when the context
+// changes, e.g. after a device reset).
 static __device__ __align__(256) float g_noalloc_partials[NVFP4_NOALLOC_MAX_PARTIALS];
 
-// First call on the current device: look up the array's device address.
+// First call in the current context: look up the array's device address.
 nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
   std::lock_guard<std::mutex> lock(g_mutex);
   if (st->noalloc_partials == nullptr) {

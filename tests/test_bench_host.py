@@ -101,7 +101,8 @@ def test_clock_summary_window_and_reasons():
     assert c["samples"] == 13 and c["window"].startswith("whole run")
     assert c["reasons"] == ["sw_power_cap", "sw_thermal_slowdown"]
     s.samples = [(1.0, "garbage"), (1.1, "0, N/A, N/A")]
-    assert s.summary(0.0, 2.0) is None
+    c = s.summary(0.0, 2.0)                                          # no usable sample
+    assert c["sm_mhz"] is None and c["samples"] == 0 and "error" in c
 
 
 def test_clock_sample_uses_nvidia_smi_timestamp():
