@@ -274,6 +274,46 @@ nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf
                                      int64_t ffn, int64_t k,
                                      nvfp4_stream_t stream);
 
+/* Workspace bytes of nvfp4_gemm_swiglu_quant_dynamic: bf16 h [m][ffn]
+ * (256-byte padded) and one partial maximum per GEMM CTA. 0 for bad sizes. */
+size_t nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(int64_t m, int64_t ffn);
+
+/*
+ * nvfp4_gemm_swiglu_quant_dynamic — as nvfp4_gemm_swiglu_quant, but h is
+ * quantized with its own dynamic global (g_h = 2688 / max|h| over the whole
+ * [m][ffn] tensor, as nvfp4_quantize derives it), so no calibration is
+ * needed: the W4A4 MLP of the recipe (news §03: every linear layer NVFP4)
+ * with the activation quantized on the fly like any other. A global over
+ * the whole of h is only known once all of h exists, so h is written once in
+ * bf16 (to the workspace) by the GEMM epilogue, which also records max|h| per
+ * CTA; the quantizer then reduces those maxima to g_h exactly as it reduces
+ * an amax pass's and quantizes h (no separate amax pass over h, no bf16
+ * gate/up output). Computes, bit for bit,
+ *   Y  = nvfp4_gemm(A, B) in bf16 (gate and up halves),
+ *   h  = nvfp4_silu_mul(Y),
+ *   (h_codes, h_sf, h_global_out) = nvfp4_quantize(h)   [dynamic global]
+ * with two launches (GEMM, quantizer) on `stream`.
+ *   A, B       as nvfp4_gemm_swiglu_quant (B rows interleaved in blocks of 128).
+ *   h_codes    device [m][ffn/2] bytes, 16-byte aligned.
+ *   h_sf       device nvfp4_sf_bytes(m, ffn) bytes, 16-byte aligned.
+ *   h_global_out  device FP32 scalar: receives g_h.
+ *   workspace  device scratch of at least
+ *              nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(m, ffn) bytes,
+ *              256-byte aligned, caller-owned, no initialisation needed; after
+ *              the call its first m*ffn*2 bytes hold h in bf16 (row-major,
+ *              leading dimension ffn).
+ *   ffn % 128 == 0, k % 32 == 0.
+ * Errors: INVALID_ARG (null pointer, bad size, short workspace), MISALIGNED,
+ * UNSUPPORTED (ffn % 128, k % 32, sizes >= 2^31), CUDA.
+ */
+nvfp4_status nvfp4_gemm_swiglu_quant_dynamic(const uint8_t* a_codes, const uint8_t* a_sf,
+                                             const float* a_global, const uint8_t* b_codes,
+                                             const uint8_t* b_sf, const float* b_global,
+                                             uint8_t* h_codes, uint8_t* h_sf,
+                                             float* h_global_out, int64_t m, int64_t ffn,
+                                             int64_t k, void* workspace,
+                                             size_t workspace_bytes, nvfp4_stream_t stream);
+
 /*
  * nvfp4_fuse_group_scales — global-scale repair of a fused module group
  * (news §03: a serving kernel fuses several GDN linear layers into one GEMM;

@@ -52,6 +52,11 @@
 // SwiGLU expression, h rounded to bf16) and quantizes h to NVFP4 with a
 // calibrated static global using the quantizer's arithmetic, writing codes
 // and swizzled scales of h instead of the 2*ffn-wide bf16 output.
+// A second fused mode (dynamic global of h) writes h in bf16 with the same
+// TMA-store epilogue as the plain GEMM (128 of the tile's 256 columns) and
+// one max|h| per CTA, which the quantizer then reduces to h's global exactly
+// as it reduces the amax pass's partials: the output is that of the unfused
+// chain (GEMM -> bf16 gate/up -> silu*mul -> dynamic quantization of h).
 // Launched with programmatic stream serialisation: barrier set-up and
 // tensor-memory allocation overlap the previous kernel in the stream; the
 // producer and the epilogue wait for it before touching global memory, except
@@ -122,15 +127,21 @@ struct Params {
   void* y;
   int64_t ldy;
   int y_fp32;
-  // fused SwiGLU + quantize mode (y unused): h = [M][ffn], ffn = N / 2
+  // Fused SwiGLU modes (h = [M][ffn], ffn = N / 2; y unused):
+  //   kFusedQuantStatic  h quantized to NVFP4 with the static h_global
+  //   kFusedBf16Amax     h written in bf16 through the tensor map of Y, and
+  //                      max|h| over this CTA's tiles to h_partials[CTA]
   int fused;
   const float* h_global;   // static global of h
   uint8_t* h_codes;        // [M][ffn/2]
   uint8_t* h_sf;           // swizzled scales of [M][ffn]
   int64_t h_atoms;         // 512-byte atoms per 128-row block = ffn / 64
   int m_pad;               // rows of the scale buffer = ceil(M/128)*128
+  float* h_partials;       // [gridDim.x] per-CTA max|h| (kFusedBf16Amax)
   int early_w;             // B may be read before the previous kernel finishes
 };
+
+enum : int { kPlain = 0, kFusedQuantStatic = 1, kFusedBf16Amax = 2 };
 
 // Band rasterization: consecutive tiles walk GROUP_M M-tiles down one N band,
 // so the pairs resident at one time share A and B tiles in L2, and a band's
@@ -244,6 +255,34 @@ __device__ __forceinline__ uint32_t swiglu_quant_block(const uint32_t* g, const 
   return sc;
 }
 
+// 32 columns of h for the kFusedBf16Amax mode: gate/up accumulators -> bf16
+// (as the plain GEMM stores them) -> SwiGLU -> bf16 h, staged like
+// stage_bf16; `amax` accumulates max|h| over the values written.
+__device__ __forceinline__ void stage_h(uint32_t chunk, int row, const uint32_t (&g)[32],
+                                        const uint32_t (&u)[32], float alpha, float& amax) {
+  const uint32_t base = chunk + row * 64;
+  const int sw = (row >> 1) & 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float h[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const int c = q * 8 + 2 * e + i;
+        const float gb = __bfloat162float(__float2bfloat16_rn(__uint_as_float(g[c]) * alpha));
+        const float ub = __bfloat162float(__float2bfloat16_rn(__uint_as_float(u[c]) * alpha));
+        h[i] = act::swiglu(gb, ub);
+      }
+      const __nv_bfloat162 b2 = __floats2bfloat162_rn(h[0], h[1]);
+      amax = fmaxf(amax, fmaxf(fabsf(__low2float(b2)), fabsf(__high2float(b2))));
+      w[e] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    ptx::st_shared_v4(base + ((q ^ sw) << 4), w[0], w[1], w[2], w[3]);
+  }
+}
+
 // Tensor-memory columns of scale buffer `buf`: A's 16, then B's 32.
 __device__ __forceinline__ uint32_t sfa_cols(uint32_t tmem, uint32_t buf) {
   return tmem + SF_COL + buf * SF_BUF_COLS;
@@ -296,6 +335,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* drain_sf = sf_full + NSF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
+  uint32_t* h_max = tmem_holder + 2;  // kFusedBf16Amax: max|h| bits over the CTA
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -317,12 +357,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     ptx::mbar_init(drain_sf, NUM_SF_WARPS);
     *abort_flag = 0u;
+    *h_max = 0u;
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tmA);
     ptx::tma_prefetch_desc(&tmB);
     ptx::tma_prefetch_desc(&tmSFA);
     ptx::tma_prefetch_desc(&tmSFB);
-    if (!p.fused) ptx::tma_prefetch_desc(&tmY);
+    if (p.fused != kFusedQuantStatic) ptx::tma_prefetch_desc(&tmY);
   }
   if (warp == 1) {
     ptx::tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -494,7 +535,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // -------------------------------------------------------------- epilogue --
     ptx::grid_dep_wait();  // globals from earlier kernels; Y / h may still be in use
     float* rtab = reinterpret_cast<float*>(smem + RTAB_OFF);
-    if (p.fused) {
+    if (p.fused == kFusedQuantStatic) {
       // E4M3 code -> g_h / dec(code), as the quantizer tabulates it
       const float gh = __ldg(p.h_global);
       const int t = threadIdx.x - EPI_WARP0 * 32;
@@ -526,12 +567,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ++nchunk;
     };
     uint32_t acc_phase = 0;
+    float h_amax = 0.0f;  // kFusedBf16Amax: max|h| over this thread's values
     for (int t = pair; t < num_tiles; t += num_pairs) {
       int mb, nb;
       tile_coords(t, p, mb, nb);
       if (!wait_bounded(tmem_full, acc_phase, ab, kFaultEpilogue)) break;
       ptx::tc_fence_after();
-      if (p.fused) {
+      if (p.fused == kFusedBf16Amax) {
+        // gate columns [64 half, +64) and the matching up columns (+128) ->
+        // 64 bf16 h columns of 32 rows, two TMA-stored chunks
+        uint32_t g0[32], g1[32], u0[32], u1[32];
+        const uint32_t lb = tmem + (static_cast<uint32_t>(q * 32) << 16) + 64u * half;
+        ptx::tc_ld_32x32b_x32(lb + 0u, g0);
+        ptx::tc_ld_32x32b_x32(lb + 32u, g1);
+        ptx::tc_ld_32x32b_x32(lb + 128u, u0);
+        ptx::tc_ld_32x32b_x32(lb + 160u, u1);
+        ptx::tc_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive_cluster(release);
+        acc_phase ^= 1u;
+        const int row0 = mb * BM + static_cast<int>(rank) * HALF + q * 32;
+        if (row0 >= p.M) continue;  // rows past M inside are zero (h = 0) and clipped
+        const int hc0 = nb * 128 + 64 * half;
+        emit([&](uint32_t b) { stage_h(b, lane, g0, u0, alpha, h_amax); }, hc0, row0);
+        emit([&](uint32_t b) { stage_h(b, lane, g1, u1, alpha, h_amax); }, hc0 + 32, row0);
+        continue;
+      }
+      if (p.fused == kFusedQuantStatic) {
         // gate columns [64 half, +64) and the matching up columns (+128)
         uint32_t g0[32], g1[32], u0[32], u1[32];
         const uint32_t lb = tmem + (static_cast<uint32_t>(q * 32) << 16) + 64u * half;
@@ -597,6 +660,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
     if (lane == 0) ptx::bulk_wait_group_all();  // stores done before the CTA can exit
+    if (p.fused == kFusedBf16Amax) {
+      // one partial max per CTA (order-free, so the global that the
+      // quantizer derives from the partials does not depend on timing);
+      // every epilogue warp gets here, also after an abort
+      const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(h_amax));
+      if (lane == 0) atomicMax(h_max, wm);
+      asm volatile("bar.sync 1, %0;" ::"n"(32 * NUM_EPI_WARPS) : "memory");
+      if (threadIdx.x == EPI_WARP0 * 32) p.h_partials[blockIdx.x] = __uint_as_float(*h_max);
+    }
   }
 
   ptx::tc_fence_before();

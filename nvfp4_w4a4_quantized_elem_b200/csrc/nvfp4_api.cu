@@ -274,6 +274,18 @@ nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
   return NVFP4_OK;
 }
 
+// The quantizer kernel over a.rows x a.k (arguments checked, occupancy
+// known): one resident wave at most, launched to overlap its predecessor.
+nvfp4_status quantizer_launch(const nvfp4::quant::QuantArgs& a, DeviceState* st, cudaStream_t s) {
+  using namespace nvfp4::quant;
+  const int64_t n_tasks = ceil_div(a.rows, 128) * 32 * ceil_div(ceil_div(a.k, 64), kAtomsPerTask);
+  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
+  const int64_t cap = static_cast<int64_t>(st->sms) * st->quant_per_sm;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return launch_pdl(quantize_kernel, static_cast<unsigned>(blocks), kQuantThreads, 0, s, 1u, a);
+}
+
 // Dynamic or static NVFP4 quantization of x (arguments already checked):
 // the amax pass (dynamic only, x above kSelfAmaxBytes) into `partials` (at
 // most max_parts CTAs), then the quantizer, launched to overlap the amax
@@ -307,11 +319,7 @@ nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx
   a.codes = codes;
   a.sf = sf;
   a.global_out = global_out;
-  int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
-  const int64_t cap = static_cast<int64_t>(st->sms) * st->quant_per_sm;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  return launch_pdl(quantize_kernel, static_cast<unsigned>(blocks), kQuantThreads, 0, s, 1u, a);
+  return quantizer_launch(a, st, s);
 }
 
 }  // namespace
@@ -562,7 +570,7 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
 nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                          const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes,
                          const uint8_t* b_sf, int64_t m, int64_t n, int64_t k,
-                         nvfp4::gemm::Params p, cudaStream_t stream) {
+                         nvfp4::gemm::Params p, cudaStream_t stream, int* grid_out = nullptr) {
   using namespace nvfp4::gemm;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
   std::memset(&tmY, 0, sizeof tmY);
@@ -574,8 +582,11 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
     return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFA, a_sf, m, k, 1u)) return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFB, b_sf, n, k, 2u)) return e;
-  if (!p.fused)
+  if (p.fused == kPlain) {
     if (nvfp4_status e = encode_y(enc, &tmY, p.y, m, n, p.ldy, p.y_fp32)) return e;
+  } else if (p.fused == kFusedBf16Amax) {  // bf16 h = [m][n / 2]
+    if (nvfp4_status e = encode_y(enc, &tmY, p.y, m, n / 2, p.ldy, 0)) return e;
+  }
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!st->gemm_smem_set) {
@@ -598,6 +609,7 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   // one CTA pair (cluster of 2 SMs) per 256x256 tile at a time, persistent
   const int64_t max_pairs = st->sms / 2;
   const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  if (grid_out != nullptr) *grid_out = 2 * pairs;
   return launch_pdl(gemm_kernel, static_cast<unsigned>(2 * pairs), NUM_THREADS, SMEM_BYTES,
                     stream, 2u, tmA, tmB, tmSFA, tmSFB, tmY, p);
 }
@@ -724,7 +736,7 @@ nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf
   std::memset(&p, 0, sizeof p);
   p.a_global = a_global;
   p.b_global = b_global;
-  p.fused = 1;
+  p.fused = nvfp4::gemm::kFusedQuantStatic;
   p.h_global = h_global;
   p.h_codes = h_codes;
   p.h_sf = h_sf;
@@ -732,6 +744,77 @@ nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf
   p.m_pad = static_cast<int>(ceil_div(m, 128) * 128);
   return gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, 2 * ffn, k, p,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(int64_t m, int64_t ffn) {
+  if (m < 1 || ffn < 1) return 0;
+  return round_up(static_cast<size_t>(m) * static_cast<size_t>(ffn) * 2u, 256) +
+         static_cast<size_t>(nvfp4::quant::kMaxPartials) * sizeof(float);
+}
+
+nvfp4_status nvfp4_gemm_swiglu_quant_dynamic(const uint8_t* a_codes, const uint8_t* a_sf,
+                                             const float* a_global, const uint8_t* b_codes,
+                                             const uint8_t* b_sf, const float* b_global,
+                                             uint8_t* h_codes, uint8_t* h_sf, float* h_global_out,
+                                             int64_t m, int64_t ffn, int64_t k, void* workspace,
+                                             size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (!a_codes || !a_sf || !a_global || !b_codes || !b_sf || !b_global || !h_codes || !h_sf ||
+      !h_global_out || !workspace)
+    return NVFP4_ERR_INVALID_ARG;
+  if (m < 1 || ffn < 1 || k < 1) return NVFP4_ERR_INVALID_ARG;
+  if (ffn % 128 != 0 || k % 32 != 0 || m >= (int64_t{1} << 31) || 2 * ffn >= (int64_t{1} << 31) ||
+      k >= (int64_t{1} << 31))
+    return NVFP4_ERR_UNSUPPORTED;
+  if (!aligned(a_codes, 16) || !aligned(b_codes, 16) || !aligned(a_sf, 16) || !aligned(b_sf, 16) ||
+      !aligned(h_codes, 16) || !aligned(h_sf, 16) || !aligned(a_global, 4) ||
+      !aligned(b_global, 4) || !aligned(h_global_out, 4) || !aligned(workspace, 256))
+    return NVFP4_ERR_MISALIGNED;
+  if (workspace_bytes < nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(m, ffn))
+    return NVFP4_ERR_INVALID_ARG;
+  using namespace nvfp4::quant;
+  // 32-bit task index of the quantizer over h
+  if (ceil_div(m, 128) * 32 * ceil_div(ceil_div(ffn, 64), kAtomsPerTask) >= (int64_t{1} << 31))
+    return NVFP4_ERR_UNSUPPORTED;
+  int dev;
+  DeviceState* st;
+  if (nvfp4_status e = current_device(&dev, &st)) return e;
+  if (nvfp4_status e = quant_occupancy(st)) return e;
+  PFN_cuTensorMapEncodeTiled_v12000 enc;
+  if (nvfp4_status e = get_encoder(&enc)) return e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // workspace: [bf16 h, m x ffn][per-CTA max|h|]
+  uint16_t* h = static_cast<uint16_t*>(workspace);
+  float* partials = reinterpret_cast<float*>(
+      static_cast<uint8_t*>(workspace) +
+      round_up(static_cast<size_t>(m) * static_cast<size_t>(ffn) * 2u, 256));
+  nvfp4::gemm::Params p;
+  std::memset(&p, 0, sizeof p);
+  p.a_global = a_global;
+  p.b_global = b_global;
+  p.fused = nvfp4::gemm::kFusedBf16Amax;
+  p.y = h;
+  p.ldy = ffn;
+  p.h_partials = partials;
+  int grid = 0;
+  if (nvfp4_status e = gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, 2 * ffn, k, p, s,
+                                   &grid))
+    return e;
+  if (grid > kMaxPartials) return NVFP4_ERR_UNSUPPORTED;  // cannot happen: grid <= SM count
+  // the quantizer reduces the GEMM's per-CTA maxima to h's global, as it
+  // reduces an amax pass's, and quantizes h (launched to overlap the GEMM's
+  // tail; it waits for the GEMM before reading anything)
+  QuantArgs a;
+  a.x = h;
+  a.rows = m;
+  a.k = ffn;
+  a.ldx = ffn;
+  a.global_in = nullptr;
+  a.partials = partials;
+  a.nparts = grid;
+  a.codes = h_codes;
+  a.sf = h_sf;
+  a.global_out = h_global_out;
+  return quantizer_launch(a, st, s);
 }
 
 nvfp4_status nvfp4_fuse_group_scales(int n_modules, const int64_t* rows_per_module, int64_t k,

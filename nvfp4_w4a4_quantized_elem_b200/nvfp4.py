@@ -30,6 +30,7 @@ EXPORTS = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_quantize_workspace_by
            "nvfp4_quantize", "nvfp4_quantize_noalloc", "nvfp4_calibrate_global",
            "nvfp4_gemm_workspace_bytes", "nvfp4_gemm", "nvfp4_linear_workspace_bytes",
            "nvfp4_linear", "nvfp4_gemm_swiglu_quant",
+           "nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes", "nvfp4_gemm_swiglu_quant_dynamic",
            "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault",
            "nvfp4_selftest_wait_timeout")
 
@@ -68,6 +69,9 @@ def lib() -> ctypes.CDLL:
             "nvfp4_linear_workspace_bytes": (SZ, [I64, I64, I64]),
             "nvfp4_linear": (I, [P, I64, I64, I64, P, P, P, P, I64, P, I, I64, P, SZ, P]),
             "nvfp4_gemm_swiglu_quant": (I, [P, P, P, P, P, P, P, P, P, I64, I64, I64, P]),
+            "nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes": (SZ, [I64, I64]),
+            "nvfp4_gemm_swiglu_quant_dynamic": (I, [P, P, P, P, P, P, P, P, P, I64, I64, I64,
+                                                    P, SZ, P]),
             "nvfp4_fuse_group_scales": (I, [I, P, I64, P, P, P, P, P]),
             "nvfp4_silu_mul": (I, [P, I64, I64, I64, P, I64, P]),
             "nvfp4_read_fault": (I, [P, U32P]),
@@ -249,6 +253,36 @@ def gemm_swiglu_quant(a: NVFP4Tensor, b_interleaved: NVFP4Tensor, h_global: torc
                                        _ptr(b_interleaved.global_scale), _ptr(h_global),
                                        _ptr(out.codes), _ptr(out.sf), m, ffn, k, _stream(stream))
     _check(st, "nvfp4_gemm_swiglu_quant")
+    return out
+
+
+def swiglu_quant_dynamic_workspace(m: int, ffn: int, device="cuda") -> torch.Tensor:
+    """Workspace of gemm_swiglu_quant_dynamic (bf16 h + per-CTA maxima)."""
+    nb = int(lib().nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(m, ffn))
+    return torch.empty(nb, dtype=torch.uint8, device=device)
+
+
+def gemm_swiglu_quant_dynamic(a: NVFP4Tensor, b_interleaved: NVFP4Tensor,
+                              out: NVFP4Tensor | None = None,
+                              workspace: torch.Tensor | None = None,
+                              stream: torch.cuda.Stream | None = None) -> NVFP4Tensor:
+    """nvfp4_gemm_swiglu_quant_dynamic: NVFP4 h = quantize(silu(gate) * up)
+    with h's own dynamic global (weights row-interleaved, see
+    interleave_gate_up). ``workspace`` from swiglu_quant_dynamic_workspace()
+    (allocated here when None); its first m*ffn*2 bytes hold h in bf16."""
+    if a.k != b_interleaved.k:
+        raise ValueError("k mismatch")
+    m, ffn, k = a.rows, b_interleaved.rows // 2, a.k
+    if out is None:
+        out = NVFP4Tensor.empty(m, ffn, a.codes.device)
+    if workspace is None:
+        workspace = swiglu_quant_dynamic_workspace(m, ffn, a.codes.device)
+    st = lib().nvfp4_gemm_swiglu_quant_dynamic(
+        _ptr(a.codes), _ptr(a.sf), _ptr(a.global_scale), _ptr(b_interleaved.codes),
+        _ptr(b_interleaved.sf), _ptr(b_interleaved.global_scale), _ptr(out.codes), _ptr(out.sf),
+        _ptr(out.global_scale), m, ffn, k, _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream))
+    _check(st, "nvfp4_gemm_swiglu_quant_dynamic")
     return out
 
 

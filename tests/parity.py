@@ -71,3 +71,22 @@ def gemm_check(y_gpu: torch.Tensor, y_ref: np.ndarray, row_norm: np.ndarray,
 def norms(orc, q, rows=None):
     dq = orc.dequantize(q) if rows is None else orc.dequantize_rows(q, rows)
     return np.linalg.norm(dq, axis=1)
+
+
+def assert_row_blocks_equal(orc, gpu, x_rows_bf16, blocks, g, what=""):
+    """Whole 128-row blocks of a quantized tensor against the oracle: the
+    oracle quantizes each block's rows (bf16, taken from the tensor the GPU
+    quantized) with the same global g; codes and the block's swizzled scale
+    bytes (one 128-row block is n_ka * 512 contiguous bytes) must be equal.
+    `x_rows_bf16(r0, r1)` returns rows [r0, r1) on the host."""
+    k = gpu.k
+    blk = 128 * (-(-k // 64) * 4)
+    for rb in blocks:
+        r0, r1 = 128 * rb, min(128 * rb + 128, gpu.rows)
+        q = orc.quantize(bits(x_rows_bf16(r0, r1)), global_in=np.float32(g))
+        codes = gpu.codes[r0:r1].cpu().numpy()
+        sf = gpu.sf[rb * blk:(rb + 1) * blk].cpu().numpy()
+        bad = np.argwhere(codes != q.codes)
+        assert bad.size == 0, f"{what}: block {rb}: {len(bad)} code bytes differ"
+        bad = np.flatnonzero(sf != q.sf_swizzled)
+        assert bad.size == 0, f"{what}: block {rb}: {bad.size} scale bytes differ"

@@ -151,6 +151,24 @@ def test_swiglu_quant_argument_checks(L):
     assert f(*args(h=None)) == INVALID
 
 
+def test_swiglu_quant_dynamic_argument_checks(L):
+    f = L.nvfp4_gemm_swiglu_quant_dynamic
+    need = L.nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(8, 256)
+    assert need >= 8 * 256 * 2 + 4 * 148
+    assert L.nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes(0, 256) == 0
+
+    def args(ffn=256, k=512, hg=FAKE, ws=FAKE, wsb=need):
+        return (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(hg),
+                8, ffn, k, P(ws), wsb, None)
+    assert f(*args(ffn=200, wsb=1 << 24)) == UNSUPPORTED   # ffn % 128
+    assert f(*args(k=48)) == UNSUPPORTED
+    assert f(*args(hg=None)) == INVALID
+    assert f(*args(ws=None)) == INVALID
+    assert f(*args(ws=FAKE + 16)) == MISALIGNED           # workspace: 256-byte alignment
+    assert f(*args(hg=FAKE + 2)) == MISALIGNED
+    assert f(*args(wsb=need - 1)) == INVALID                # short workspace
+
+
 def lin(L, x=FAKE, m=8, k=64, ldx=64, xg=None, wc=FAKE, wsf=FAKE, wg=FAKE, n=64, y=FAKE, yd=0,
         ldy=64, ws=FAKE, wsb=1 << 24):
     return L.nvfp4_linear(P(x), m, k, ldx, P(xg), P(wc), P(wsf), P(wg), n, P(y), yd, ldy, P(ws),

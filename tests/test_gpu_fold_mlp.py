@@ -101,7 +101,7 @@ def test_mlp32k_pipeline_full(nv, orc):
     """X 32768x5120 (5 outlier channels x30) -> gate_up W 34816x5120 ->
     silu*mul -> requantize h (dynamic global) -> down W 5120x17408, all on the
     GPU. Checks: quantized X, W, h bit-exact (h from the GPU's own silu*mul
-    output); silu*mul within 1 bf16 ulp; both GEMMs on 256 sampled rows."""
+    output); silu*mul within 1 bf16 ulp; both GEMMs on 1024 sampled rows."""
     from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
     cfg = wl.mlp32k()
     x = cfg.x()
@@ -116,7 +116,7 @@ def test_mlp32k_pipeline_full(nv, orc):
     Wd = nv.quantize(wd.cuda())
     out = nv.gemm(H, Wd)
     torch.cuda.synchronize()
-    rows = np.sort(np.random.default_rng(1).choice(cfg.m, 256, replace=False))
+    rows = np.sort(np.random.default_rng(1).choice(cfg.m, 1024, replace=False))
     ridx = torch.from_numpy(rows).cuda()
 
     qa = orc.quantize(bits(x))

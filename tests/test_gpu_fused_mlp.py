@@ -12,7 +12,7 @@ import numpy as np
 import pytest
 import torch
 
-from parity import assert_quant_equal, bits
+from parity import assert_quant_equal, assert_row_blocks_equal, bits
 
 pytestmark = pytest.mark.gpu
 
@@ -86,9 +86,58 @@ def test_swiglu_quant_mlp32k_full(nv, orc):
     torch.cuda.synchronize()
     assert torch.equal(fused.codes, ref.codes)
     assert torch.equal(fused.sf, ref.sf)
-    rows = np.sort(np.random.default_rng(3).choice(cfg.m, 128, replace=False))
-    hr = h[torch.from_numpy(rows).cuda()].cpu()
+    # whole 128-row blocks (codes and their swizzled scale bytes) vs the oracle
+    blocks = np.sort(np.random.default_rng(3).choice(cfg.m // 128, 4, replace=False))
     g = gh.cpu().numpy()[0]
-    q = orc.quantize(bits(hr), global_in=g)
-    np.testing.assert_array_equal(fused.codes[torch.from_numpy(rows).cuda()].cpu().numpy(), q.codes)
+    assert_row_blocks_equal(orc, fused, lambda r0, r1: h[r0:r1].cpu(), blocks, g, "fused h")
+    assert nv.read_fault() == 0
+
+
+@pytest.mark.parametrize("m,ffn,k", [(65, 384, 512), (300, 256, 288), (1000, 640, 1024),
+                                     (2048, 1024, 768)])
+def test_swiglu_quant_dynamic_equals_unfused_chain(nv, orc, m, ffn, k):
+    """Dynamic global of h: the fused GEMM (bf16 h + per-CTA max|h|) followed
+    by the quantizer equals GEMM -> silu*mul -> dynamic quantize bit for bit,
+    and the oracle's dynamic quantization of the same bf16 h."""
+    x = gaussian(m, k, 11 * m)
+    w = gaussian(2 * ffn, k, 13 * ffn, 0.02)
+    A = nv.quantize(x.cuda())
+    Bi = nv.quantize(nv.interleave_gate_up(w.cuda()))
+    h = unfused_h(nv, A, Bi, ffn)
+    ref = nv.quantize(h)
+    ws = nv.swiglu_quant_dynamic_workspace(m, ffn)
+    fused = nv.gemm_swiglu_quant_dynamic(A, Bi, workspace=ws)
+    torch.cuda.synchronize()
+    h_ws = ws[:m * ffn * 2].view(torch.bfloat16).view(m, ffn)
+    assert torch.equal(h_ws, h)
+    assert torch.equal(fused.codes, ref.codes)
+    assert torch.equal(fused.sf, ref.sf)
+    assert torch.equal(fused.global_scale, ref.global_scale)
+    assert_quant_equal(fused, orc.quantize(bits(h.cpu())), "fused dynamic vs oracle")
+    # a second call into the same workspace (stale partials and h) agrees
+    fused2 = nv.gemm_swiglu_quant_dynamic(A, Bi, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(fused2.codes, ref.codes) and torch.equal(fused2.sf, ref.sf)
+    assert nv.read_fault() == 0
+
+
+def test_swiglu_quant_dynamic_mlp32k_full(nv, orc):
+    """The 32K-token MLP's gate_up with the dynamic global of h: equal to the
+    unfused chain bit for bit; g_h equal to the oracle's 2688 / max|h| over
+    the whole h; whole 128-row blocks equal to the oracle's quantization."""
+    from nvfp4_w4a4_quantized_elem_b200 import workloads as wl
+    cfg = wl.mlp32k()
+    A = nv.quantize(cfg.x().cuda())
+    Bi = nv.quantize(nv.interleave_gate_up(cfg.w_gate_up().cuda()))
+    h = unfused_h(nv, A, Bi, cfg.ffn)
+    ref = nv.quantize(h)
+    fused = nv.gemm_swiglu_quant_dynamic(A, Bi)
+    torch.cuda.synchronize()
+    assert torch.equal(fused.codes, ref.codes)
+    assert torch.equal(fused.sf, ref.sf)
+    h_host = h.cpu()
+    g = orc.global_from_amax(orc.tensor_amax(bits(h_host)))
+    assert fused.global_scale.cpu().numpy()[0].view(np.uint32) == np.float32(g).view(np.uint32)
+    blocks = np.sort(np.random.default_rng(4).choice(cfg.m // 128, 4, replace=False))
+    assert_row_blocks_equal(orc, fused, lambda r0, r1: h_host[r0:r1], blocks, g, "dynamic h")
     assert nv.read_fault() == 0
