@@ -365,6 +365,31 @@ nvfp4_status nvfp4_silu_mul(const void* y, int64_t m, int64_t n, int64_t ldy,
                             void* h, int64_t ldh, nvfp4_stream_t stream);
 
 /*
+ * nvfp4_selftest_gemm_stall — failure-detection self-test of the GEMM
+ * kernels themselves (no counterpart on the pages; it exists so that the
+ * time-out and abort path of the kernels that do the work can be run on a
+ * GPU without a fault). Runs nvfp4_gemm (bf16 Y, ldy = n) with two changes:
+ * every wait of the kernel gives up after `limit_ns` instead of 2 s, and
+ * the TMA producers issue nothing for the first ring stage, so that stage's
+ * barrier never completes. Every role then runs into its limit (or sees the
+ * abort another role raised), in-flight copies and tensor-core work are
+ * drained, tensor memory is freed and the kernel returns; nvfp4_read_fault
+ * then reports NVFP4_ERR_TIMEOUT with the role bits (paired kernel, m > 64:
+ * 1 producer, 2 MMA, 4 epilogue, 8 scale copies; few-token kernel, m <= 64:
+ * 16, 32, 64, 128). Y is left undefined, and for m <= 64 the workspace's
+ * reduction counters must be zeroed again before it is reused (nvfp4_gemm
+ * zeroes them itself; nvfp4_linear does not).
+ *   Arguments as nvfp4_gemm (y bf16 [m][n]); limit_ns in [1 us, 10 s].
+ * Errors: as nvfp4_gemm; INVALID_ARG for limit_ns out of range.
+ */
+nvfp4_status nvfp4_selftest_gemm_stall(const uint8_t* a_codes, const uint8_t* a_sf,
+                                       const float* a_global, const uint8_t* b_codes,
+                                       const uint8_t* b_sf, const float* b_global, void* y,
+                                       int64_t m, int64_t n, int64_t k, uint64_t limit_ns,
+                                       void* workspace, size_t workspace_bytes,
+                                       nvfp4_stream_t stream);
+
+/*
  * nvfp4_read_fault — every mbarrier wait in the GEMM kernel is bounded; on
  * expiry the kernel records a nonzero fault word, stops issuing work and
  * returns instead of hanging. This call synchronises `stream`, copies the

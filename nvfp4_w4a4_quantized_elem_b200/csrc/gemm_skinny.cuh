@@ -105,6 +105,11 @@ struct Params {
   float* partial;           // stream-K: [num_w_tiles][kMaxContrib][M][BW] FP32 slabs
   unsigned int* tile_count; // stream-K: [num_w_tiles * 4], zero before and after a launch
   int early_w;              // weights may be read before the previous kernel finishes
+  // Failure-detection self-test only (0 in every product call): the
+  // producer issues nothing for the first ring stage, so its full barrier
+  // never completes and every role's bounded wait runs into its limit.
+  int stall_first_stage;
+  uint64_t wait_limit_ns;   // per-wait limit; 0 = kWaitLimitNs
 };
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
@@ -244,6 +249,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint64_t lim = p.wait_limit_ns != 0 ? p.wait_limit_ns : kWaitLimitNs;
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
       ptx::mbar_init(&full[s], 1);
@@ -270,6 +276,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // The next kernel in the stream may be scheduled on SMs as they free up
+  // (it waits for this grid's completion before it reads anything this
+  // grid writes): a decode layer's quantizer and GEMM launches then overlap
+  // this GEMM's tail.
+  ptx::grid_dep_launch();
   const uint32_t tmem = *tmem_holder;
 
   if (warp == 0) {
@@ -303,12 +314,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       stage = static_cast<uint32_t>(npre % C::STAGES);
       phase = static_cast<uint32_t>(npre / C::STAGES);
+      bool stall = p.stall_first_stage != 0 && npre == 0;
       for (; it.sg.valid; it.next(p)) {
-        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer)) {
+        if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer, lim)) {
           aborted = true;
           break;
         }
         pending &= ~(1u << stage);
+        if (stall) {  // self-test: this stage is never filled (nothing in flight for it)
+          stall = false;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
         ptx::tma_load_2d(st, &tmW, &full[stage], it.kt * BK_BYTES, it.sg.wt * BW);
@@ -324,9 +344,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           phase ^= 1u;
         }
       }
-      if (aborted)
-        for (int s = 0; s < C::STAGES; ++s)
-          if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
+      // Let every issued copy land before the CTA can exit: after an abort
+      // (raised here or, later, by another role) nothing else waits for
+      // them; without one the MMA thread consumes the same phases, so these
+      // waits end as soon as the last copies land.
+      (void)aborted;
+      for (int s = 0; s < C::STAGES; ++s)
+        if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
     }
   } else if (warp == 1) {
     // ----------------------------------------------------------- MMA issuer --
@@ -337,14 +361,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       SegIter sg;
       for (sg.first(p); sg.valid && !aborted; sg.next(p)) {
         const int k0 = sg.k0, k1 = sg.k1;
-        if (!wait_bounded(tmem_empty, acc_phase ^ 1u, abort_flag, kFaultMma)) {
+        if (!wait_bounded(tmem_empty, acc_phase ^ 1u, abort_flag, kFaultMma, lim)) {
           aborted = true;
           break;
         }
         ptx::tc_fence_after();
         for (int kt = k0; kt < k1; ++kt) {
-          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma) ||
-              !wait_bounded(&sf_full[stage], phase, abort_flag, kFaultMma)) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma, lim) ||
+              !wait_bounded(&sf_full[stage], phase, abort_flag, kFaultMma, lim)) {
             aborted = true;
             break;
           }
@@ -387,7 +411,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         for (int kt = sg.k0; kt < sg.k1; ++kt) {
           // the stage's data having landed means its previous MMAs finished
           // (the producer waited for them), so scale buffer `stage` is free
-          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales)) {
+          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales, lim)) {
             aborted = true;
             break;
           }
@@ -436,7 +460,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         n_contrib = cta_of(static_cast<int64_t>(wt + 1) * p.num_k_tiles - 1, T, gridDim.x) -
                     c_first + 1;
       }
-      if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue)) break;
+      if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue, lim)) break;
       ptx::tc_fence_after();
       const int nl = q * 32 + lane;            // column within the weight tile
       const int n = wt * BW + nl;              // this thread's output column

@@ -139,6 +139,11 @@ struct Params {
   int m_pad;               // rows of the scale buffer = ceil(M/128)*128
   float* h_partials;       // [gridDim.x] per-CTA max|h| (kFusedBf16Amax)
   int early_w;             // B may be read before the previous kernel finishes
+  // Failure-detection self-test only (0 in every product call): the
+  // producers issue nothing for the first ring stage, so its full barrier
+  // never completes and every role's bounded wait runs into its limit.
+  int stall_first_stage;
+  uint64_t wait_limit_ns;  // per-wait limit; 0 = kWaitLimitNs
 };
 
 enum : int { kPlain = 0, kFusedQuantStatic = 1, kFusedBf16Amax = 2 };
@@ -161,6 +166,7 @@ __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int
 struct Abort {
   volatile uint32_t* local;   // this CTA's flag
   uint32_t peer_cluster;      // shared::cluster address of the peer's flag
+  uint64_t limit_ns;          // limit of one wait
 
   __device__ __forceinline__ bool raised() const { return *local != 0u; }
   __device__ __forceinline__ void raise(uint32_t who) const {
@@ -179,7 +185,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, con
   while (true) {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     if (ab.raised()) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (ptx::globaltimer_ns() - t0 > ab.limit_ns) {
       ab.raise(who);
       return false;
     }
@@ -372,9 +378,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   ptx::tc_fence_before();
   ptx::cluster_sync();  // barriers of both CTAs initialised, TMEM allocated
   ptx::tc_fence_after();
+  // Every CTA of this grid is resident: the next kernel in the stream may be
+  // scheduled on SMs as they free up (it waits for this grid's completion
+  // before it reads anything this grid writes).
+  ptx::grid_dep_launch();
   const uint32_t tmem = *tmem_holder;
   const Abort ab{abort_flag,
-                 ptx::mapa_shared(ptx::smem_u32(const_cast<uint32_t*>(abort_flag)), rank ^ 1u)};
+                 ptx::mapa_shared(ptx::smem_u32(const_cast<uint32_t*>(abort_flag)), rank ^ 1u),
+                 p.wait_limit_ns != 0 ? p.wait_limit_ns : kWaitLimitNs};
   const int num_tiles = p.num_m_blk * p.num_n_blk;
 
   if (warp == 0) {
@@ -430,12 +441,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       stage = static_cast<uint32_t>(npre % STAGES);
       phase = static_cast<uint32_t>(npre / STAGES);
+      bool stall = p.stall_first_stage != 0 && npre == 0;
       for (; it.t < num_tiles; it = next(it)) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, ab, kFaultProducer)) {
           aborted = true;
           break;
         }
         pending &= ~(1u << stage);
+        if (stall) {  // self-test: this stage is never filled (nothing in flight for it)
+          stall = false;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+          continue;
+        }
         if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
         load_a(it, stage);
         load_b(it, stage);
@@ -446,8 +466,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           phase ^= 1u;
         }
       }
-      if (aborted && leader) {
-        // let every issued copy of the pair land before the CTAs can exit
+      if (leader) {
+        // Let every issued copy of the pair land before the CTAs can exit:
+        // after an abort (raised here or, later, by another role) nothing
+        // else waits for them. Without one the MMA thread consumes the same
+        // phases, so these waits end as soon as the last copies land.
+        (void)aborted;
         for (int s = 0; s < STAGES; ++s)
           if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
       }
@@ -671,9 +695,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   }
 
+  // Neither CTA frees tensor memory or exits while the pair works: the peer
+  // may still signal this CTA's barriers (TMA completions, MMA commits,
+  // accumulator releases) or write its tensor memory. This barrier is left
+  // without a time limit on purpose: every role above reaches it within the
+  // sum of its bounded waits and drains, and a CTA that gave up on it and
+  // exited could still be addressed by its peer.
   ptx::tc_fence_before();
   __syncwarp();
-  ptx::cluster_sync();  // neither CTA frees tensor memory while the pair works
+  ptx::cluster_sync();
   ptx::tc_fence_after();
   if (warp == 1) {
     __syncwarp();

@@ -511,7 +511,7 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
                          void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
                          void* workspace, size_t workspace_bytes, bool zero_counters,
-                         int early_w, cudaStream_t s) {
+                         int early_w, cudaStream_t s, int stall = 0, uint64_t limit_ns = 0) {
   using namespace nvfp4::skinny;
   const int bnt = m <= 16 ? 16 : m <= 32 ? 32 : 64;  // callers route m <= 64 here
   CUtensorMap tmW, tmX, tmSFW, tmSFX;
@@ -538,6 +538,8 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   p.tile_count = nullptr;
   p.early_w = early_w;
   p.stream_k = 0;
+  p.stall_first_stage = stall;
+  p.wait_limit_ns = limit_ns;
   int grid = static_cast<int>(p.num_w_tiles < st->sms ? p.num_w_tiles : st->sms);
   const bool split_ok = workspace != nullptr &&
                         workspace_bytes >= skinny_workspace_bytes(m, n) && aligned(workspace, 16);
@@ -618,10 +620,16 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
 
 extern "C" {
 
-nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+}  // extern "C"
+
+namespace {
+
+// nvfp4_gemm; `stall` / `limit_ns` only for nvfp4_selftest_gemm_stall.
+nvfp4_status gemm_entry(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
                         const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
                         void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
-                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream,
+                        int stall, uint64_t limit_ns) {
   using namespace nvfp4::gemm;
   if (!a_codes || !a_sf || !a_global || !b_codes || !b_sf || !b_global || !y)
     return NVFP4_ERR_INVALID_ARG;
@@ -642,7 +650,7 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   if (m <= 64)
     return gemm_skinny(enc, st, a_codes, a_sf, a_global, b_codes, b_sf, b_global, y, y_dtype, ldy,
                        m, n, k, workspace, workspace_bytes, true, 0,
-                       reinterpret_cast<cudaStream_t>(stream));
+                       reinterpret_cast<cudaStream_t>(stream), stall, limit_ns);
 
   nvfp4::gemm::Params p;
   std::memset(&p, 0, sizeof p);
@@ -651,8 +659,33 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float
   p.y = y;
   p.ldy = ldy;
   p.y_fp32 = y_dtype;
+  p.stall_first_stage = stall;
+  p.wait_limit_ns = limit_ns;
   return gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, n, k, p,
                      reinterpret_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                        const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
+                        void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
+                        void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  return gemm_entry(a_codes, a_sf, a_global, b_codes, b_sf, b_global, y, y_dtype, ldy, m, n, k,
+                    workspace, workspace_bytes, stream, 0, 0);
+}
+
+nvfp4_status nvfp4_selftest_gemm_stall(const uint8_t* a_codes, const uint8_t* a_sf,
+                                       const float* a_global, const uint8_t* b_codes,
+                                       const uint8_t* b_sf, const float* b_global, void* y,
+                                       int64_t m, int64_t n, int64_t k, uint64_t limit_ns,
+                                       void* workspace, size_t workspace_bytes,
+                                       nvfp4_stream_t stream) {
+  if (limit_ns < 1000u || limit_ns > 10000000000ull) return NVFP4_ERR_INVALID_ARG;
+  return gemm_entry(a_codes, a_sf, a_global, b_codes, b_sf, b_global, y, 0, n, m, n, k,
+                    workspace, workspace_bytes, stream, 1, limit_ns);
 }
 
 size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {

@@ -8,7 +8,9 @@
 //
 // Both kernels wait for the previous kernel in the stream before touching
 // global memory, so they may be launched with programmatic stream
-// serialisation (the next kernel's launch then overlaps this one's tail).
+// serialisation; each lets the next kernel be scheduled as soon as it starts
+// (that kernel in turn waits for this one before it reads what this one
+// writes), so a following GEMM's set-up and weight loads can overlap it.
 // Two kernels:
 //   amax_kernel      one pass over x, one partial max per CTA (no atomics, so
 //                    the workspace needs no initialisation);
@@ -101,8 +103,8 @@ __device__ __forceinline__ uint32_t absmax_bits8(uint4 v) {
 __global__ void __launch_bounds__(kAmaxThreads)
     amax_kernel(const uint16_t* __restrict__ x, int64_t rows, int64_t k, int64_t ldx,
                 float* __restrict__ partials) {
+  ptx::grid_dep_launch();  // the next kernel may be scheduled; it waits for this one itself
   ptx::grid_dep_wait();
-  ptx::grid_dep_launch();
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
@@ -162,8 +164,8 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs a) {
+  ptx::grid_dep_launch();  // the next kernel may be scheduled; it waits for this one itself
   ptx::grid_dep_wait();    // partials / static global / x come from earlier kernels
-  ptx::grid_dep_launch();
   __shared__ float s_g;
   __shared__ float s_rtab[128];
   __shared__ uint32_t s_red[kQuantThreads / 32];
@@ -308,8 +310,8 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
 __global__ void __launch_bounds__(256)
     calibrate_kernel(const float* __restrict__ partials, int nparts, float* running_amax,
                      float* global_out) {
-  ptx::grid_dep_wait();
   ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
   __shared__ uint32_t s_red[8];
   uint32_t m = 0;
   for (int i = threadIdx.x; i < nparts; i += blockDim.x) m = max(m, __float_as_uint(partials[i]));

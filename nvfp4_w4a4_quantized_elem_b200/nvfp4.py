@@ -32,7 +32,7 @@ EXPORTS = ("nvfp4_status_string", "nvfp4_sf_bytes", "nvfp4_quantize_workspace_by
            "nvfp4_linear", "nvfp4_gemm_swiglu_quant",
            "nvfp4_gemm_swiglu_quant_dynamic_workspace_bytes", "nvfp4_gemm_swiglu_quant_dynamic",
            "nvfp4_fuse_group_scales", "nvfp4_silu_mul", "nvfp4_read_fault",
-           "nvfp4_selftest_wait_timeout")
+           "nvfp4_selftest_wait_timeout", "nvfp4_selftest_gemm_stall")
 
 _lib = None
 _lock = threading.Lock()
@@ -76,6 +76,8 @@ def lib() -> ctypes.CDLL:
             "nvfp4_silu_mul": (I, [P, I64, I64, I64, P, I64, P]),
             "nvfp4_read_fault": (I, [P, U32P]),
             "nvfp4_selftest_wait_timeout": (I, [ctypes.c_uint64, P]),
+            "nvfp4_selftest_gemm_stall": (I, [P, P, P, P, P, P, P, I64, I64, I64, ctypes.c_uint64,
+                                              P, SZ, P]),
         }
         for name, (res, args) in sigs.items():
             fn = getattr(L, name)
@@ -345,7 +347,24 @@ def selftest_wait_timeout(limit_ns: int = 1_000_000,
     """nvfp4_selftest_wait_timeout: make one bounded wait give up on the GPU
     (read_fault() then returns 256)."""
     _check(lib().nvfp4_selftest_wait_timeout(limit_ns, _stream(stream)),
-           "nvfp4_selftest_wait_timeout")
+           "nvfp4_selftest_wait_timeout", "nvfp4_selftest_gemm_stall")
+
+
+def selftest_gemm_stall(a: NVFP4Tensor, b: NVFP4Tensor, limit_ns: int = 1_000_000,
+                        workspace: torch.Tensor | None = None,
+                        stream: torch.cuda.Stream | None = None) -> None:
+    """nvfp4_selftest_gemm_stall: run the GEMM kernel for these operands
+    with its first ring stage never filled and every wait limited to
+    ``limit_ns``; the kernel gives up and returns (read_fault() then returns
+    the role bits that timed out)."""
+    m, n, k = a.rows, b.rows, a.k
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=a.codes.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().nvfp4_selftest_gemm_stall(_ptr(a.codes), _ptr(a.sf), _ptr(a.global_scale),
+                                           _ptr(b.codes), _ptr(b.sf), _ptr(b.global_scale),
+                                           _ptr(y), m, n, k, limit_ns, _ptr(workspace), ws_bytes,
+                                           _stream(stream)),
+           "nvfp4_selftest_gemm_stall")
 
 
 def linear_workspace_bytes(m: int, n: int, k: int) -> int:

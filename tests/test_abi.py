@@ -207,3 +207,8 @@ def test_selftest_limit_checks(L):
     assert f(0, None) == INVALID
     assert f(999, None) == INVALID
     assert f(20_000_000_000, None) == INVALID
+    g = L.nvfp4_selftest_gemm_stall
+    args = lambda lim: (P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), 256, 256,
+                        512, lim, None, 0, None)
+    assert g(*args(999)) == INVALID
+    assert g(*args(20_000_000_000)) == INVALID
