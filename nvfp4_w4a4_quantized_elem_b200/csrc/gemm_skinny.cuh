@@ -287,7 +287,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       uint32_t stage = 0, phase = 0, pending = 0, pending_parity = 0;
-      bool aborted = false;
       WorkIter it;
       it.start(p);
       // The first ring's worth of stages needs no empty-slot wait. With
@@ -317,7 +316,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool stall = p.stall_first_stage != 0 && npre == 0;
       for (; it.sg.valid; it.next(p)) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, abort_flag, kFaultProducer, lim)) {
-          aborted = true;
           break;
         }
         pending &= ~(1u << stage);
@@ -348,7 +346,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // (raised here or, later, by another role) nothing else waits for
       // them; without one the MMA thread consumes the same phases, so these
       // waits end as soon as the last copies land.
-      (void)aborted;
       for (int s = 0; s < C::STAGES; ++s)
         if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
     }

@@ -393,7 +393,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       uint32_t pending = 0, pending_parity = 0;  // stages loaded, not yet seen free
-      bool aborted = false;
       // issue order: (tile, k-tile) pairs of this CTA pair
       struct Item {
         int t, kt, mb, nb;
@@ -444,7 +443,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       bool stall = p.stall_first_stage != 0 && npre == 0;
       for (; it.t < num_tiles; it = next(it)) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, ab, kFaultProducer)) {
-          aborted = true;
           break;
         }
         pending &= ~(1u << stage);
@@ -471,7 +469,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // after an abort (raised here or, later, by another role) nothing
         // else waits for them. Without one the MMA thread consumes the same
         // phases, so these waits end as soon as the last copies land.
-        (void)aborted;
         for (int s = 0; s < STAGES; ++s)
           if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
       }
