@@ -144,9 +144,35 @@ struct Params {
   // never completes and every role's bounded wait runs into its limit.
   int stall_first_stage;
   uint64_t wait_limit_ns;  // per-wait limit; 0 = kWaitLimitNs
+  // Split-K (plain mode only; 1 = off): the K range of every tile is cut
+  // into `split` slices, one work unit each. A unit stores its FP32 partial
+  // tile to `partial`; per epilogue region (32 rows x 128 columns of one
+  // CTA) the last slice to count itself in on `tile_count` sums all slices'
+  // partials in slice order, writes Y and resets the counter.
+  int split;
+  float* partial;             // [tiles][split][2 CTAs][8 regions][32 x 128] FP32
+  unsigned int* tile_count;   // [tiles][2 CTAs][8 regions], zero before and after
 };
 
 enum : int { kPlain = 0, kFusedQuantStatic = 1, kFusedBf16Amax = 2 };
+
+// A work unit: one tile's k-tiles [k0, k1) (the whole K range without split).
+struct Unit {
+  int tile, slice, k0, k1;
+};
+
+__device__ __forceinline__ Unit unit_of(int u, const Params& p) {
+  Unit w;
+  w.tile = u / p.split;
+  w.slice = u - w.tile * p.split;
+  w.k0 = w.slice * p.num_k_tiles / p.split;
+  w.k1 = (w.slice + 1) * p.num_k_tiles / p.split;
+  return w;
+}
+
+constexpr int kRegionFloats = 32 * 128;  // one epilogue warp's part of a tile
+constexpr int kMaxSplitK = 4;            // slices per tile at most (host-checked)
+constexpr int kMinSliceKTiles = 16;      // k-tiles per slice at least (host-checked)
 
 // Band rasterization: consecutive tiles walk GROUP_M M-tiles down one N band,
 // so the pairs resident at one time share A and B tiles in L2, and a band's
@@ -289,6 +315,34 @@ __device__ __forceinline__ void stage_h(uint32_t chunk, int row, const uint32_t 
   }
 }
 
+// Split-K: one lane's 32 consecutive columns of a region (8 float4, 32
+// float4 apart in the slab layout) summed over the S slices in slice order;
+// every slice's loads are issued before the first add (one L2 round trip).
+template <int S>
+__device__ __forceinline__ void sum_slices(const float4* src, int64_t slice_stride4,
+                                           uint32_t (&acc)[32]) {
+  float4 v[S][8];
+#pragma unroll
+  for (int sl = 0; sl < S; ++sl)
+#pragma unroll
+    for (int c = 0; c < 8; ++c) v[sl][c] = __ldcg(src + 32 * c + sl * slice_stride4);
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    float4 a = v[0][c];
+#pragma unroll
+    for (int sl = 1; sl < S; ++sl) {
+      a.x += v[sl][c].x;
+      a.y += v[sl][c].y;
+      a.z += v[sl][c].z;
+      a.w += v[sl][c].w;
+    }
+    acc[4 * c] = __float_as_uint(a.x);
+    acc[4 * c + 1] = __float_as_uint(a.y);
+    acc[4 * c + 2] = __float_as_uint(a.z);
+    acc[4 * c + 3] = __float_as_uint(a.w);
+  }
+}
+
 // Tensor-memory columns of scale buffer `buf`: A's 16, then B's 32.
 __device__ __forceinline__ uint32_t sfa_cols(uint32_t tmem, uint32_t buf) {
   return tmem + SF_COL + buf * SF_BUF_COLS;
@@ -387,23 +441,29 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                  ptx::mapa_shared(ptx::smem_u32(const_cast<uint32_t*>(abort_flag)), rank ^ 1u),
                  p.wait_limit_ns != 0 ? p.wait_limit_ns : kWaitLimitNs};
   const int num_tiles = p.num_m_blk * p.num_n_blk;
+  const int num_units = num_tiles * p.split;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer --
     if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       uint32_t pending = 0, pending_parity = 0;  // stages loaded, not yet seen free
-      // issue order: (tile, k-tile) pairs of this CTA pair
+      // issue order: (unit, k-tile) pairs of this CTA pair
       struct Item {
-        int t, kt, mb, nb;
+        int t, kt, k1, mb, nb;
       };
       auto first = [&](int t) {
-        Item it{t, 0, 0, 0};
-        if (t < num_tiles) tile_coords(t, p, it.mb, it.nb);
+        Item it{t, 0, 0, 0, 0};
+        if (t < num_units) {
+          const Unit w = unit_of(t, p);
+          it.kt = w.k0;
+          it.k1 = w.k1;
+          tile_coords(w.tile, p, it.mb, it.nb);
+        }
         return it;
       };
       auto next = [&](Item it) {
-        if (++it.kt == p.num_k_tiles) it = first(it.t + num_pairs);
+        if (++it.kt == it.k1) it = first(it.t + num_pairs);
         return it;
       };
       // the even CTA's barrier counts both CTAs' bytes of a stage
@@ -428,7 +488,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // halves are requested before the grid-dependency wait.
       int npre = 0;
       if (p.early_w) {
-        for (Item w = it; npre < STAGES && w.t < num_tiles; ++npre, w = next(w)) {
+        for (Item w = it; npre < STAGES && w.t < num_units; ++npre, w = next(w)) {
           if (leader) ptx::mbar_arrive_expect_tx(&full[npre], 2 * STAGE_BYTES);
           load_b(w, static_cast<uint32_t>(npre));
         }
@@ -441,7 +501,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       stage = static_cast<uint32_t>(npre % STAGES);
       phase = static_cast<uint32_t>(npre / STAGES);
       bool stall = p.stall_first_stage != 0 && npre == 0;
-      for (; it.t < num_tiles; it = next(it)) {
+      for (; it.t < num_units; it = next(it)) {
         if (!wait_bounded(&empty[stage], phase ^ 1u, ab, kFaultProducer)) {
           break;
         }
@@ -479,8 +539,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t smem_base = ptx::smem_u32(smem);
       uint32_t stage = 0, phase = 0, acc_phase = 0;
       bool aborted = false;
-      for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
-        for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+      for (int t = pair; t < num_units && !aborted; t += num_pairs) {
+        const Unit w = unit_of(t, p);
+        for (int kt = w.k0; kt < w.k1; ++kt) {
           if (!wait_bounded(&full[stage], phase, ab, kFaultMma) ||
               !wait_bounded(&sf_full[stage], phase, ab, kFaultMma)) {
             aborted = true;
@@ -489,7 +550,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ptx::tc_fence_after();
           const uint32_t sa = smem_base + stage * STAGE_BYTES;
           const uint32_t sb = sa + A_BYTES;
-          if (kt == 0) {
+          if (kt == w.k0) {
             // the accumulator must have been drained by both epilogues
             if (!wait_bounded(tmem_empty, acc_phase ^ 1u, ab, kFaultMma)) {
               aborted = true;
@@ -504,7 +565,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const uint64_t adesc = ptx::smem_desc(sa + 32u * j, 16, 1024, 2);
             const uint64_t bdesc = ptx::smem_desc(sb + 32u * j, 16, 1024, 2);
             ptx::tc_mma_nvf4_pair(tmem + ACC_COL, adesc, bdesc, IDESC, tsfa + 4u * j,
-                                  tsfb + 8u * j, (kt | j) != 0 ? 1u : 0u);
+                                  tsfb + 8u * j, (kt != w.k0 || j != 0) ? 1u : 0u);
           }
           // frees the stage in both CTAs, and with it the stage's scale buffer
           ptx::tc_commit_pair_mc(&empty[stage], 0x3);
@@ -528,8 +589,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t smem_base = ptx::smem_u32(smem);
       uint32_t stage = 0, phase = 0;
       bool aborted = false;
-      for (int t = pair; t < num_tiles && !aborted; t += num_pairs) {
-        for (int kt = 0; kt < p.num_k_tiles; ++kt) {
+      for (int t = pair; t < num_units && !aborted; t += num_pairs) {
+        const Unit w = unit_of(t, p);
+        for (int kt = w.k0; kt < w.k1; ++kt) {
           // The stage's data having landed also means the MMAs of its previous
           // use finished (the producer waited for them before reloading it),
           // so scale buffer `stage` is free: no wait on the MMA thread here.
@@ -589,9 +651,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     };
     uint32_t acc_phase = 0;
     float h_amax = 0.0f;  // kFusedBf16Amax: max|h| over this thread's values
-    for (int t = pair; t < num_tiles; t += num_pairs) {
+    for (int t = pair; t < num_units; t += num_pairs) {
+      const Unit unit = unit_of(t, p);
       int mb, nb;
-      tile_coords(t, p, mb, nb);
+      tile_coords(unit.tile, p, mb, nb);
       if (!wait_bounded(tmem_full, acc_phase, ab, kFaultEpilogue)) break;
       ptx::tc_fence_after();
       if (p.fused == kFusedBf16Amax) {
@@ -662,8 +725,61 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       acc_phase ^= 1u;
 
       const int row0 = mb * BM + static_cast<int>(rank) * HALF + q * 32;  // this warp's rows
-      if (row0 >= p.M) continue;  // warp-uniform; rows past M inside are clipped by the TMA
       const int col0 = nb * BN + half * 128;
+      if (p.split > 1) {
+        // this slice's partial -> its slab; the region's last slice sums all
+        // slabs in slice order (whichever slice that is) and writes Y
+        const int region = static_cast<int>(rank) * 8 + (warp - EPI_WARP0);
+        const int64_t slab_stride = int64_t{16} * kRegionFloats;  // one slice of a tile
+        float* const base = p.partial + int64_t{unit.tile} * p.split * slab_stride +
+                            int64_t{region} * kRegionFloats;
+        float4* mine = reinterpret_cast<float4*>(base + unit.slice * slab_stride) + lane;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          __stcg(mine + 32 * c, make_float4(__uint_as_float(r0[4 * c]), __uint_as_float(r0[4 * c + 1]),
+                                            __uint_as_float(r0[4 * c + 2]),
+                                            __uint_as_float(r0[4 * c + 3])));
+          __stcg(mine + 32 * (8 + c),
+                 make_float4(__uint_as_float(r1[4 * c]), __uint_as_float(r1[4 * c + 1]),
+                             __uint_as_float(r1[4 * c + 2]), __uint_as_float(r1[4 * c + 3])));
+          __stcg(mine + 32 * (16 + c),
+                 make_float4(__uint_as_float(r2[4 * c]), __uint_as_float(r2[4 * c + 1]),
+                             __uint_as_float(r2[4 * c + 2]), __uint_as_float(r2[4 * c + 3])));
+          __stcg(mine + 32 * (24 + c),
+                 make_float4(__uint_as_float(r3[4 * c]), __uint_as_float(r3[4 * c + 1]),
+                             __uint_as_float(r3[4 * c + 2]), __uint_as_float(r3[4 * c + 3])));
+        }
+        __threadfence();
+        __syncwarp();
+        unsigned int* cnt = p.tile_count + unit.tile * 16 + region;
+        uint32_t last = 0;
+        if (lane == 0) last = atomicAdd(cnt, 1u) == static_cast<unsigned>(p.split - 1);
+        last = __shfl_sync(0xFFFFFFFFu, last, 0);
+        if (!last) continue;
+        __threadfence();
+        if (row0 < p.M) {
+          // 32 columns at a time: all slices' loads first, then the adds
+          for (int cc = 0; cc < 4; ++cc) {
+            uint32_t acc[32];
+            const float4* src = reinterpret_cast<const float4*>(base) + lane + 32 * (8 * cc);
+            switch (p.split) {
+              case 2: sum_slices<2>(src, slab_stride / 4, acc); break;
+              case 3: sum_slices<3>(src, slab_stride / 4, acc); break;
+              default: sum_slices<kMaxSplitK>(src, slab_stride / 4, acc); break;
+            }
+            if (!p.y_fp32) {
+              emit([&](uint32_t b) { stage_bf16(b, lane, acc, alpha); }, col0 + 32 * cc, row0);
+            } else {
+              emit([&](uint32_t b) { stage_f32(b, lane, acc, 0, alpha); }, col0 + 32 * cc, row0);
+              emit([&](uint32_t b) { stage_f32(b, lane, acc, 16, alpha); }, col0 + 32 * cc + 16,
+                   row0);
+            }
+          }
+        }
+        if (lane == 0) *cnt = 0u;  // ready for the next call
+        continue;
+      }
+      if (row0 >= p.M) continue;  // warp-uniform; rows past M inside are clipped by the TMA
       if (!p.y_fp32) {
         emit([&](uint32_t b) { stage_bf16(b, lane, r0, alpha); }, col0 + 0, row0);
         emit([&](uint32_t b) { stage_bf16(b, lane, r1, alpha); }, col0 + 32, row0);

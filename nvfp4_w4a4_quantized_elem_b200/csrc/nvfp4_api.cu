@@ -189,6 +189,36 @@ size_t skinny_workspace_bytes(int64_t m, int64_t n) {
                                        nvfp4::skinny::BW * sizeof(float);
 }
 
+// Split-K of the paired kernel (nvfp4::gemm, m > 64): when the 256x256 tiles
+// cannot occupy half the CTA pairs, the K range is cut into S slices (at most
+// kMaxSplitK, each at least kMinSliceKTiles k-tiles) so that tiles x S units
+// occupy the pairs; e.g. 20 tiles of a 256-token 17408 -> 5120 layer run as
+// 60 units instead of 20. Workspace: counters (16 per tile), then the FP32
+// partial tiles. The workspace bytes depend on the shape only (the largest
+// S any device could use); the launch picks S from the SM count.
+constexpr int64_t kSplitMaxTiles = 64;
+int64_t paired_tiles(int64_t m, int64_t n) {
+  return ceil_div(m, nvfp4::gemm::BM) * ceil_div(n, nvfp4::gemm::BN);
+}
+int paired_split_cap(int64_t m, int64_t n, int64_t k) {
+  using namespace nvfp4::gemm;
+  const int64_t kt = ceil_div(k, BK);
+  if (m <= 64 || paired_tiles(m, n) > kSplitMaxTiles || kt < 2 * kMinSliceKTiles) return 1;
+  return static_cast<int>(kt / kMinSliceKTiles < kMaxSplitK ? kt / kMinSliceKTiles : kMaxSplitK);
+}
+size_t paired_counter_bytes(int64_t tiles) {
+  return round_up(static_cast<size_t>(tiles) * 16 * sizeof(unsigned int), 256);
+}
+size_t paired_split_bytes(int64_t tiles, int split) {
+  return paired_counter_bytes(tiles) + static_cast<size_t>(tiles) * static_cast<size_t>(split) *
+                                           16 * nvfp4::gemm::kRegionFloats * sizeof(float);
+}
+int paired_split(int sms, int64_t m, int64_t n, int64_t k) {
+  const int cap = paired_split_cap(m, n, k);
+  const int64_t by_pairs = (sms / 2) / paired_tiles(m, n);
+  return static_cast<int>(by_pairs < cap ? by_pairs : cap);
+}
+
 // Stream-K grid of a few-token GEMM: G CTAs sharing the W x KT iterations,
 // at most kMaxSplits per weight tile, shrunk until no tile has more than
 // kMaxContrib contributing CTAs (each has a slab slot). 0 = no split: whole
@@ -424,10 +454,12 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k, int6
 }
 
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
-  (void)k;
-  if (m < 1 || n < 1) return 0;
+  if (m < 1 || n < 1 || k < 1) return 0;
   // few-token GEMMs share the work stream-K fashion: counters and FP32 slabs
-  return m <= 64 ? skinny_workspace_bytes(m, n) : 0;
+  if (m <= 64) return skinny_workspace_bytes(m, n);
+  // paired kernel with few tiles: split-K counters and FP32 partial tiles
+  const int cap = paired_split_cap(m, n, k);
+  return cap >= 2 ? paired_split_bytes(paired_tiles(m, n), cap) : 0;
 }
 
 }  // extern "C"
@@ -569,10 +601,15 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
 
 // The paired-CTA kernel (cta_group::2, 256x256 tiles): M, N, K, tile counts
 // and tensor maps filled in here; output / fused fields come in `p`.
+// Split-K (plain mode) when `workspace` holds at least paired_split_bytes for
+// the S this device uses; its counters are zeroed here when `zero_counters`,
+// else the caller guarantees they are zero (every call leaves them so).
 nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                          const uint8_t* a_codes, const uint8_t* a_sf, const uint8_t* b_codes,
                          const uint8_t* b_sf, int64_t m, int64_t n, int64_t k,
-                         nvfp4::gemm::Params p, cudaStream_t stream, int* grid_out = nullptr) {
+                         nvfp4::gemm::Params p, cudaStream_t stream, int* grid_out = nullptr,
+                         void* workspace = nullptr, size_t workspace_bytes = 0,
+                         bool zero_counters = true) {
   using namespace nvfp4::gemm;
   CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
   std::memset(&tmY, 0, sizeof tmY);
@@ -608,21 +645,29 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   p.num_k_tiles = static_cast<int>(ceil_div(k, BK));
   const int64_t tiles = static_cast<int64_t>(p.num_m_blk) * p.num_n_blk;
   if (tiles >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;
-  // one CTA pair (cluster of 2 SMs) per 256x256 tile at a time, persistent
+  p.split = 1;
+  if (p.fused == kPlain && workspace != nullptr && aligned(workspace, 16)) {
+    const int sk = paired_split(st->sms, m, n, k);
+    if (sk >= 2 && workspace_bytes >= paired_split_bytes(tiles, sk)) {
+      p.split = sk;
+      p.tile_count = static_cast<unsigned int*>(workspace);
+      p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
+                                           paired_counter_bytes(tiles));
+      if (zero_counters &&
+          cudaMemsetAsync(workspace, 0, paired_counter_bytes(tiles), stream) != cudaSuccess) {
+        cudaGetLastError();
+        return NVFP4_ERR_CUDA;
+      }
+    }
+  }
+  const int64_t units = tiles * p.split;
+  // one CTA pair (cluster of 2 SMs) per 256x256 work unit at a time, persistent
   const int64_t max_pairs = st->sms / 2;
-  const int pairs = static_cast<int>(tiles < max_pairs ? tiles : max_pairs);
+  const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
   if (grid_out != nullptr) *grid_out = 2 * pairs;
   return launch_pdl(gemm_kernel, static_cast<unsigned>(2 * pairs), NUM_THREADS, SMEM_BYTES,
                     stream, 2u, tmA, tmB, tmSFA, tmSFB, tmY, p);
 }
-
-}  // namespace
-
-extern "C" {
-
-}  // extern "C"
-
-namespace {
 
 // nvfp4_gemm; `stall` / `limit_ns` only for nvfp4_selftest_gemm_stall.
 nvfp4_status gemm_entry(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
@@ -662,7 +707,8 @@ nvfp4_status gemm_entry(const uint8_t* a_codes, const uint8_t* a_sf, const float
   p.stall_first_stage = stall;
   p.wait_limit_ns = limit_ns;
   return gemm_paired(enc, st, a_codes, a_sf, b_codes, b_sf, m, n, k, p,
-                     reinterpret_cast<cudaStream_t>(stream));
+                     reinterpret_cast<cudaStream_t>(stream), nullptr, workspace, workspace_bytes,
+                     true);
 }
 
 }  // namespace
@@ -690,7 +736,7 @@ nvfp4_status nvfp4_selftest_gemm_stall(const uint8_t* a_codes, const uint8_t* a_
 
 size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   if (m < 1 || n < 1 || k < 32 || k % 32 != 0) return 0;
-  size_t b = m <= 64 ? round_up(skinny_workspace_bytes(m, n), 256) : 0;
+  size_t b = round_up(nvfp4_gemm_workspace_bytes(m, n, k), 256);  // split / stream-K
   b += round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);  // codes
   b += round_up(nvfp4_sf_bytes(m, k), 256);                                // scales
   b += 256;                                                                // global
@@ -720,9 +766,9 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   PFN_cuTensorMapEncodeTiled_v12000 enc;
   if (nvfp4_status e = get_encoder(&enc)) return e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // workspace: [counters + slabs (m <= 64)][codes][scales][global][partials]
+  // workspace: [counters + slabs (split work)][codes][scales][global][partials]
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  const size_t split_bytes = m <= 64 ? round_up(skinny_workspace_bytes(m, n), 256) : 0;
+  const size_t split_bytes = round_up(nvfp4_gemm_workspace_bytes(m, n, k), 256);
   uint8_t* a_codes = w + split_bytes;
   uint8_t* a_sf = a_codes + round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);
   float* a_global = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(m, k), 256));
@@ -741,7 +787,8 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   p.ldy = ldy;
   p.y_fp32 = y_dtype;
   p.early_w = 1;
-  return gemm_paired(enc, st, a_codes, a_sf, w_codes, w_sf, m, n, k, p, s);
+  return gemm_paired(enc, st, a_codes, a_sf, w_codes, w_sf, m, n, k, p, s, nullptr,
+                     split_bytes ? w : nullptr, split_bytes, false);
 }
 
 nvfp4_status nvfp4_gemm_swiglu_quant(const uint8_t* a_codes, const uint8_t* a_sf,

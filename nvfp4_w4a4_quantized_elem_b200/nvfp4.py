@@ -347,7 +347,7 @@ def selftest_wait_timeout(limit_ns: int = 1_000_000,
     """nvfp4_selftest_wait_timeout: make one bounded wait give up on the GPU
     (read_fault() then returns 256)."""
     _check(lib().nvfp4_selftest_wait_timeout(limit_ns, _stream(stream)),
-           "nvfp4_selftest_wait_timeout", "nvfp4_selftest_gemm_stall")
+           "nvfp4_selftest_wait_timeout")
 
 
 def selftest_gemm_stall(a: NVFP4Tensor, b: NVFP4Tensor, limit_ns: int = 1_000_000,

@@ -114,3 +114,28 @@ def test_gemm_few_tokens_split_k(nv, orc, m):
     """Few-token path with K split across CTAs (N = 1000: 8 weight tiles,
     so most of the GPU works on K slices) and ragged token counts."""
     run_case(nv, orc, gaussian(m, 2048, 7 * m), gaussian(1000, 2048, 11, 0.02), what=f"split m={m}")
+
+
+@pytest.mark.parametrize("m,n,k", [(200, 1024, 8192), (300, 512, 12288), (256, 256, 16384),
+                                   (65, 2560, 8192)])
+def test_gemm_paired_split_k(nv, orc, m, n, k):
+    """Paired kernel with K cut into 2-4 slices (few 256x256 tiles, long K):
+    within the tolerance in both output dtypes, bit-identical from run to
+    run (the last slice of each region sums the partials in slice order,
+    whichever slice finishes last), and nvfp4_linear (which takes the same
+    split from its workspace) gives the same bits as nvfp4_gemm."""
+    x, w = gaussian(m, k, 3 * m + k), gaussian(n, k, 5 * n + k, 0.02)
+    assert nv.gemm_workspace_bytes(m, n, k) > 0
+    run_case(nv, orc, x, w, what=f"split-K {m}x{n}x{k}", workspaces=(True,))
+    qa, qb = orc.quantize(bits(x)), orc.quantize(bits(w))
+    A, B = upload(qa), upload(qb)
+    ws = torch.zeros(nv.gemm_workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    ys = [nv.gemm(A, B, out_dtype=torch.float32, workspace=ws) for _ in range(3)]
+    torch.cuda.synchronize()
+    assert all(torch.equal(ys[0], y) for y in ys[1:])
+    y_lin = nv.linear(x.cuda(), nv.quantize(w.cuda()), out_dtype=torch.float32)
+    y_gemm = nv.gemm(nv.quantize(x.cuda()), nv.quantize(w.cuda()), out_dtype=torch.float32,
+                     workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(y_lin, y_gemm)
+    assert nv.read_fault() == 0
