@@ -124,10 +124,12 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t rows, int64_t k, int64_t ldx,
  * Arguments, layouts, results and errors are those of nvfp4_quantize (minus
  * the workspace pair). Additionally:
  *   - NVFP4_ERR_UNSUPPORTED if the amax pass would need more than
- *     NVFP4_NOALLOC_MAX_PARTIALS CTAs. Its grid is capped at one resident
- *     wave (SM count x resident amax CTAs per SM, from an occupancy query):
- *     296 on a 148-SM B200 today; the cap is checked on every call, so a
- *     device or build with a larger wave gets this error, never an overrun.
+ *     NVFP4_NOALLOC_MAX_PARTIALS CTAs. It launches one CTA per 16384
+ *     elements (256-thread CTAs) for x of at most 16 MiB, so at most 512,
+ *     and for larger x one resident wave of 1024-thread CTAs (SM count x
+ *     resident CTAs per SM, from an occupancy query: 296 on a 148-SM B200);
+ *     the bound is checked on every call, so a device or build with a
+ *     larger wave gets this error, never an overrun.
  *   - The first call in a CUDA context looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current); make that first call
  *     before any stream capture. The library keys the address on the

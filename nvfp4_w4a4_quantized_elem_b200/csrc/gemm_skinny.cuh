@@ -58,14 +58,19 @@ constexpr int BK_BYTES = BK / 2;
 constexpr int NUM_THREADS = 256;
 constexpr int SF_WARP0 = 2;       // warps 2, 3 copy scales
 constexpr int EPI_WARP0 = 4;      // warps 4..7 drain the accumulator
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_BUF_COLS = 48;  // per scale buffer: weights 16, tokens up to 32
+// Half of an SM per CTA (tensor memory, shared memory, registers), so that
+// a CTA of the next decode layer's GEMM can start on the same SM while this
+// one drains: its first weight tiles then stream during this one's tail.
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t SF_BUF_COLS = 32;  // per scale buffer: weights 16, tokens 16
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
-constexpr size_t kSmemBudget = 220 * 1024;
+// dynamic shared memory per CTA such that two CTAs fit in an SM's 228 KiB
+// (each CTA also holds 1 KiB reserved by the system)
+constexpr size_t kSmemPerCta = 114 * 1024;
 constexpr int kMaxSplits = 8;     // stream-K: at most this many CTAs per weight tile
 constexpr int kMaxContrib = kMaxSplits + 1;  // contributor slots per tile (host-checked)
-constexpr int kSumTokens = 16;    // tokens summed per round of slab loads
+constexpr int kSumTokens = 8;     // tokens summed per round of slab loads
 
 enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, kFaultScales = 128u };
 
@@ -79,12 +84,14 @@ struct Cfg {
   static constexpr int SFB_BYTES = 2048 * SFB_BLOCKS;
   static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int STAGES_FIT = static_cast<int>(kSmemBudget / STAGE_BYTES);
+  static constexpr int STAGES_FIT = static_cast<int>((kSmemPerCta - 1024 - 512) / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
-  // one tensor-memory scale buffer per stage, after the BNT-column accumulator
+  static_assert(SMEM_BYTES <= kSmemPerCta, "two CTAs per SM");
+  // two BNT-column accumulators (a segment's MMAs run while the epilogue
+  // drains the previous segment), then one scale buffer per stage
   static constexpr int NSF = STAGES;
-  static constexpr uint32_t SF_COL = BNT < 32 ? 32u : static_cast<uint32_t>(BNT);
+  static constexpr uint32_t SF_COL = 2u * BNT;
   static_assert(SF_COL + NSF * SF_BUF_COLS <= TMEM_COLS, "scale buffers exceed tensor memory");
   static constexpr uint32_t SFB_COLS = 4u * SFB_BLOCKS;     // per K = 64 step
   // kind::mxf4nvf4, E2M1 x E2M1, both K-major, N = BNT, UE4M3 scales, M = 128
@@ -229,7 +236,7 @@ __device__ __forceinline__ void sum_slabs(const float* col, int64_t slab, int m0
 }
 
 template <int BNT>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+__global__ void __launch_bounds__(NUM_THREADS, 2)
     skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                   const __grid_constant__ CUtensorMap tmSFW,
                   const __grid_constant__ CUtensorMap tmSFX, const Params p) {
@@ -239,9 +246,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::STAGES * C::STAGE_BYTES);
   uint64_t* empty = full + C::STAGES;
-  uint64_t* tmem_full = empty + C::STAGES;
-  uint64_t* tmem_empty = tmem_full + 1;
-  uint64_t* drain = tmem_empty + 1;
+  uint64_t* tmem_full = empty + C::STAGES;   // [2]: one per accumulator
+  uint64_t* tmem_empty = tmem_full + 2;      // [2]
+  uint64_t* drain = tmem_empty + 2;
   uint64_t* sf_full = drain + 1;
   uint64_t* drain_sf = sf_full + C::NSF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
@@ -255,8 +262,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
     }
-    ptx::mbar_init(tmem_full, 1);
-    ptx::mbar_init(tmem_empty, 4);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&tmem_full[b], 1);
+      ptx::mbar_init(&tmem_empty[b], 4);
+    }
     ptx::mbar_init(drain, 1);
     for (int b = 0; b < C::NSF; ++b) {
       ptx::mbar_init(&sf_full[b], 2);
@@ -353,16 +362,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ----------------------------------------------------------- MMA issuer --
     if (lane == 0) {
       const uint32_t smem_base = ptx::smem_u32(smem);
-      uint32_t stage = 0, phase = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, acc_phase = 0, buf = 0;  // acc_phase: bit per buffer
       bool aborted = false;
       SegIter sg;
       for (sg.first(p); sg.valid && !aborted; sg.next(p)) {
         const int k0 = sg.k0, k1 = sg.k1;
-        if (!wait_bounded(tmem_empty, acc_phase ^ 1u, abort_flag, kFaultMma, lim)) {
+        if (!wait_bounded(&tmem_empty[buf], ((acc_phase >> buf) & 1u) ^ 1u, abort_flag, kFaultMma,
+                          lim)) {
           aborted = true;
           break;
         }
         ptx::tc_fence_after();
+        const uint32_t dacc = tmem + buf * static_cast<uint32_t>(BNT);
         for (int kt = k0; kt < k1; ++kt) {
           if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma, lim) ||
               !wait_bounded(&sf_full[stage], phase, abort_flag, kFaultMma, lim)) {
@@ -378,7 +389,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int j = 0; j < 4; ++j) {
             const uint64_t adesc = ptx::smem_desc(sa + 32u * j, 16, 1024, 2);
             const uint64_t bdesc = ptx::smem_desc(sb + 32u * j, 16, 1024, 2);
-            ptx::tc_mma_nvf4(tmem, adesc, bdesc, C::IDESC, tsfa + 4u * j, tsfb + C::SFB_COLS * j,
+            ptx::tc_mma_nvf4(dacc, adesc, bdesc, C::IDESC, tsfa + 4u * j, tsfb + C::SFB_COLS * j,
                              (kt != k0 || j != 0) ? 1u : 0u);
           }
           ptx::tc_commit(&empty[stage]);  // frees the stage and its scale buffer
@@ -388,8 +399,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
         if (aborted) break;
-        ptx::tc_commit(tmem_full);
-        acc_phase ^= 1u;
+        ptx::tc_commit(&tmem_full[buf]);
+        acc_phase ^= 1u << buf;
+        buf ^= 1u;
       }
       if (aborted) {
         ptx::tc_commit(drain);
@@ -445,7 +457,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     ptx::grid_dep_wait();  // the globals come from earlier kernels; Y may be in use
     const int q = warp & 3;  // tensor-memory lane quarter (warps 4..7 -> 0..3)
     const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase = 0, buf = 0;  // acc_phase: bit per accumulator
     const int64_t T = static_cast<int64_t>(p.num_w_tiles) * p.num_k_tiles;
     SegIter sg;
     for (sg.first(p); sg.valid; sg.next(p)) {
@@ -457,12 +469,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         n_contrib = cta_of(static_cast<int64_t>(wt + 1) * p.num_k_tiles - 1, T, gridDim.x) -
                     c_first + 1;
       }
-      if (!wait_bounded(tmem_full, acc_phase, abort_flag, kFaultEpilogue, lim)) break;
+      if (!wait_bounded(&tmem_full[buf], (acc_phase >> buf) & 1u, abort_flag, kFaultEpilogue, lim))
+        break;
       ptx::tc_fence_after();
       const int nl = q * 32 + lane;            // column within the weight tile
       const int n = wt * BW + nl;              // this thread's output column
       const bool n_ok = n < p.N;
-      const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t lane_base =
+          tmem + (static_cast<uint32_t>(q * 32) << 16) + buf * static_cast<uint32_t>(BNT);
       // slab of this (tile, contributor): [M][BW]
       float* slab = whole ? nullptr
                           : p.partial + (static_cast<int64_t>(wt) * kMaxContrib +
@@ -495,8 +509,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(tmem_empty);
-      acc_phase ^= 1u;
+      if (lane == 0) ptx::mbar_arrive(&tmem_empty[buf]);
+      acc_phase ^= 1u << buf;
+      buf ^= 1u;
       if (!whole) {
         // count this contributor in for these 32 columns; the last one sums
         // the tile's slabs in contributor order (= k order)

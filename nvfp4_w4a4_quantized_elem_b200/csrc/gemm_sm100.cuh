@@ -101,7 +101,6 @@ constexpr int NSF = STAGES;                   // tensor-memory scale buffers, on
 constexpr uint32_t SF_COL = 256;              // NSF x 48 columns: [A 16 | B 32]
 constexpr uint32_t SF_BUF_COLS = 48;
 static_assert(SF_COL + NSF * SF_BUF_COLS <= TMEM_COLS, "scale buffers exceed tensor memory");
-constexpr int GROUP_M = 16;                   // raster: 16 M-tiles per band
 constexpr int EPI_CHUNK_BYTES = 32 * 64;      // 32 rows x 64 bytes, 64-byte swizzle
 constexpr int EPI_WARP_BYTES = 2 * EPI_CHUNK_BYTES;
 constexpr int EPI_OFF = STAGES * STAGE_BYTES;  // staging tiles after the ring
@@ -152,6 +151,8 @@ struct Params {
   int split;
   float* partial;             // [tiles][split][2 CTAs][8 regions][32 x 128] FP32
   unsigned int* tile_count;   // [tiles][2 CTAs][8 regions], zero before and after
+  int raster_n;               // bands of N-tiles (1) or of M-tiles (0)
+  int group;                  // tiles per band (>= 1)
 };
 
 enum : int { kPlain = 0, kFusedQuantStatic = 1, kFusedBf16Amax = 2 };
@@ -174,19 +175,25 @@ constexpr int kRegionFloats = 32 * 128;  // one epilogue warp's part of a tile
 constexpr int kMaxSplitK = 4;            // slices per tile at most (host-checked)
 constexpr int kMinSliceKTiles = 16;      // k-tiles per slice at least (host-checked)
 
-// Band rasterization: consecutive tiles walk GROUP_M M-tiles down one N band,
-// so the pairs resident at one time share A and B tiles in L2, and a band's
-// A rows (16 x 256 rows) stay in L2 while B streams past them once per band.
-// With 8-tile bands the 89 MB gate_up weight was re-read from DRAM 16 times
-// (1.7 GB of DRAM reads for 184 MB of operands).
+// Band rasterization: consecutive tiles walk down a band of `group` tiles of
+// one operand (M-tiles when !raster_n, N-tiles when raster_n) and then step
+// along the other, so the pairs resident at one time share operand tiles in
+// L2 and the band's rows of its operand stay in L2 while the other operand
+// streams past once per band. The host sizes the band so that it fits in
+// L2: a whole operand of at most ~48 MB is kept resident (the other read
+// once), else the band is cut to ~48 MB of A. (Fixed 16-tile bands re-read
+// the 89 MB gate_up weight 8 times and the down projection's A 3 times.)
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
-  const int per_group = GROUP_M * p.num_n_blk;
+  const int nb_band = p.raster_n ? p.num_n_blk : p.num_m_blk;  // tiles along the band's side
+  const int nb_walk = p.raster_n ? p.num_m_blk : p.num_n_blk;
+  const int per_group = p.group * nb_walk;
   const int group = t / per_group;
-  const int first_m = group * GROUP_M;
-  const int gsize = min(p.num_m_blk - first_m, GROUP_M);
+  const int first = group * p.group;
+  const int gsize = min(nb_band - first, p.group);
   const int r = t - group * per_group;
-  mb = first_m + r % gsize;
-  nb = r / gsize;
+  const int band = first + r % gsize, walk = r / gsize;
+  mb = p.raster_n ? walk : band;
+  nb = p.raster_n ? band : walk;
 }
 
 struct Abort {

@@ -270,16 +270,26 @@ nvfp4_status quant_occupancy(DeviceState* st) {
 // (the contiguous path is flat over elements, the strided one a warp per
 // row), at most one resident wave. Sizing by rows alone starved few-row
 // inputs.
-int64_t amax_blocks(int64_t rows, int64_t k, int64_t ldx, const DeviceState* st) {
+int64_t amax_blocks(int64_t rows, int64_t k, int64_t ldx, const DeviceState* st,
+                    int threads = nvfp4::quant::kAmaxThreads) {
   using namespace nvfp4::quant;
-  const int64_t per_block = (ldx == k) ? static_cast<int64_t>(kAmaxThreads) * 8 * 8
-                                       : static_cast<int64_t>(kAmaxThreads / 32);
+  const int64_t per_block = (ldx == k) ? static_cast<int64_t>(threads) * 8 * 8
+                                       : static_cast<int64_t>(threads / 32);
   const int64_t units = (ldx == k) ? rows * k : rows;
   int64_t blocks = ceil_div(units, per_block);
-  const int64_t cap = static_cast<int64_t>(st->sms) * st->amax_per_sm;
+  const int64_t cap = static_cast<int64_t>(st->sms) * st->amax_per_sm *
+                      (kAmaxThreads / threads);
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return blocks;
+}
+
+// CTA size of the amax pass: small inputs (a decode step's tokens) run in
+// 256-thread CTAs, which fit on an SM next to a running few-token GEMM CTA
+// (half an SM), so the pass need not wait for that GEMM's CTAs to exit.
+constexpr int64_t kSmallAmaxBytes = int64_t{16} << 20;
+int amax_threads(int64_t rows, int64_t k) {
+  return rows * k * 2 <= kSmallAmaxBytes ? 256 : nvfp4::quant::kAmaxThreads;
 }
 
 // Scratch of nvfp4_quantize_noalloc: the amax pass's per-CTA partial maxima.
@@ -308,7 +318,9 @@ nvfp4_status noalloc_scratch(DeviceState* st, float** out) {
 // known): one resident wave at most, launched to overlap its predecessor.
 nvfp4_status quantizer_launch(const nvfp4::quant::QuantArgs& a, DeviceState* st, cudaStream_t s) {
   using namespace nvfp4::quant;
-  const int64_t n_tasks = ceil_div(a.rows, 128) * 32 * ceil_div(ceil_div(a.k, 64), kAtomsPerTask);
+  const int64_t n_kc = ceil_div(ceil_div(a.k, 64), kAtomsPerTask);
+  const int64_t n_tasks =
+      (a.skip_pad && a.rows < 32) ? a.rows * n_kc : ceil_div(a.rows, 128) * 32 * n_kc;
   int64_t blocks = ceil_div(n_tasks, kQuantThreads / 32);
   const int64_t cap = static_cast<int64_t>(st->sms) * st->quant_per_sm;
   if (blocks > cap) blocks = cap;
@@ -323,7 +335,7 @@ nvfp4_status quantizer_launch(const nvfp4::quant::QuantArgs& a, DeviceState* st,
 nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx,
                              const float* global_in, uint8_t* codes, uint8_t* sf,
                              float* global_out, float* partials, int64_t max_parts,
-                             DeviceState* st, cudaStream_t s) {
+                             DeviceState* st, cudaStream_t s, bool skip_pad = false) {
   using namespace nvfp4::quant;
   const int64_t n_tasks = ceil_div(rows, 128) * 32 * ceil_div(ceil_div(k, 64), kAtomsPerTask);
   if (n_tasks >= (int64_t{1} << 31)) return NVFP4_ERR_UNSUPPORTED;  // 32-bit task index
@@ -331,11 +343,12 @@ nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx
   static_assert(kSelfAmaxBytes == NVFP4_ONE_PASS_MAX_BYTES, "one-pass bound of nvfp4.h");
   int nparts = 0;  // dynamic mode with nparts == 0: the quantizer takes the max itself
   if (global_in == nullptr && rows * k * 2 > kSelfAmaxBytes) {
-    const int64_t blocks = amax_blocks(rows, k, ldx, st);
+    const int threads = amax_threads(rows, k);
+    const int64_t blocks = amax_blocks(rows, k, ldx, st, threads);
     if (blocks > max_parts) return NVFP4_ERR_UNSUPPORTED;
     nparts = static_cast<int>(blocks);
-    amax_kernel<<<nparts, kAmaxThreads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
-                                                partials);
+    amax_kernel<<<nparts, threads, 0, s>>>(static_cast<const uint16_t*>(x), rows, k, ldx,
+                                           partials);
     if (nvfp4_status e = launch_status()) return e;
   }
   QuantArgs a;
@@ -349,6 +362,7 @@ nvfp4_status quantize_launch(const void* x, int64_t rows, int64_t k, int64_t ldx
   a.codes = codes;
   a.sf = sf;
   a.global_out = global_out;
+  a.skip_pad = skip_pad ? 1 : 0;
   return quantizer_launch(a, st, s);
 }
 
@@ -660,6 +674,27 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
       }
     }
   }
+  // band rasterization (tile_coords): keep a whole operand of at most
+  // kL2BandBytes resident and stream the other once; else bands of A rows
+  // of about that size (B is then read once per band)
+  {
+    const int64_t kL2BandBytes = int64_t{48} << 20;
+    const int64_t a_bytes = m * (k / 2), b_bytes = n * (k / 2);
+    const int64_t a_tile_bytes = int64_t{BM} * (k / 2);
+    if (b_bytes <= kL2BandBytes && b_bytes <= a_bytes) {
+      p.raster_n = 1;
+      p.group = p.num_n_blk;
+    } else if (a_bytes <= kL2BandBytes) {
+      p.raster_n = 0;
+      p.group = p.num_m_blk;
+    } else {
+      int64_t g = kL2BandBytes / a_tile_bytes;
+      if (g < 8) g = 8;
+      if (g > p.num_m_blk) g = p.num_m_blk;
+      p.raster_n = 0;
+      p.group = static_cast<int>(g);
+    }
+  }
   const int64_t units = tiles * p.split;
   // one CTA pair (cluster of 2 SMs) per 256x256 work unit at a time, persistent
   const int64_t max_pairs = st->sms / 2;
@@ -773,8 +808,10 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   uint8_t* a_sf = a_codes + round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);
   float* a_global = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(m, k), 256));
   float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a_global) + 256);
+  // the quantized X is private to this call: its padding rows' scales are
+  // not written (only the GEMM reads them, against zero-filled codes)
   if (nvfp4_status e = quantize_launch(x, m, k, ldx, x_global, a_codes, a_sf, a_global, partials,
-                                       nvfp4::quant::kMaxPartials, st, s))
+                                       nvfp4::quant::kMaxPartials, st, s, true))
     return e;
   if (m <= 64)
     return gemm_skinny(enc, st, a_codes, a_sf, a_global, w_codes, w_sf, w_global, y, y_dtype, ldy,
@@ -894,6 +931,7 @@ nvfp4_status nvfp4_gemm_swiglu_quant_dynamic(const uint8_t* a_codes, const uint8
   a.codes = h_codes;
   a.sf = h_sf;
   a.global_out = h_global_out;
+  a.skip_pad = 0;
   return quantizer_launch(a, st, s);
 }
 

@@ -158,6 +158,11 @@ struct QuantArgs {
   uint8_t* codes;
   uint8_t* sf;
   float* global_out;
+  // 1: scales of the padding rows [rows, 128) of a tensor of fewer than 32
+  // rows are not written (a caller-private buffer only the GEMM reads; its
+  // padding rows multiply zero-filled codes): a decode step's few tokens
+  // then need rows x (k/256) warp tasks instead of 32 x (k/256).
+  int skip_pad;
 };
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
@@ -230,7 +235,7 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_kernel(const QuantArgs
   const int64_t n_rb = (a.rows + 127) / 128;
   const int64_t n_ka = (a.k + 63) / 64;  // 512-byte atoms per 128-row block
   const int64_t n_kc = (n_ka + kAtomsPerTask - 1) / kAtomsPerTask;
-  const int64_t n_tasks = n_rb * 32 * n_kc;
+  const int64_t n_tasks = (a.skip_pad && a.rows < 32) ? a.rows * n_kc : n_rb * 32 * n_kc;
   const int grp = lane >> 3;  // row group: row l + 32*grp
   const int j = lane & 7;     // 16-byte chunk of the row's 128-byte atom slice
   const int64_t half_k = a.k >> 1;

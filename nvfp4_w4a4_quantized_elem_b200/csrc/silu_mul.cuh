@@ -13,10 +13,19 @@ namespace act {
 
 constexpr int kThreads = 256;
 
-// silu(g) * u in FP32 with explicitly rounded steps, shared by the
-// standalone kernel and the fused GEMM epilogue so both give the same bits.
+// silu(g) * u in FP32, shared by the standalone kernel and the fused GEMM
+// epilogues so all of them give the same bits. The exponential and the
+// division are the hardware's fast forms (__expf, __fdividef: a few FP32 ulp),
+// far inside the bf16 rounding of h that follows (h stays within one bf16
+// ulp of the FP64 value); in the fused gate_up epilogue the IEEE forms cost
+// ~4x the issue slots of this expression, per element of h. Below g = -80,
+// 1 + exp(-g) leaves __fdividef's operand range (2^126) and exp(g) is no
+// longer a normal number for __expf; there silu(g) = g e^g / (1 + e^g) equals
+// g e^g in FP32, taken with the accurate expf.
 __device__ __forceinline__ float swiglu(float g, float u) {
-  return __fmul_rn(__fdiv_rn(g, __fadd_rn(1.0f, expf(-g))), u);
+  const float s = g < -80.0f ? __fmul_rn(g, expf(g))
+                             : __fdividef(g, __fadd_rn(1.0f, __expf(-g)));
+  return __fmul_rn(s, u);
 }
 
 // h = bf16(silu(gate) * up), gate = y[:, :n], up = y[:, n:2n]; one warp per

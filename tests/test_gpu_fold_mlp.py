@@ -97,6 +97,25 @@ def test_silu_mul_parity(nv, orc):
     assert torch.all((got - ref).abs() <= ulp)
 
 
+def test_silu_mul_extremes(nv, orc):
+    """silu*mul over the whole useful range of the gate, bf16 values from
+    -128 to 128 (every value the cast gives there, both signs of up): the
+    fast exponential and division and the large-negative branch stay within
+    one bf16 ulp of the FP64 oracle, zeros and subnormals included."""
+    gate = torch.linspace(-128.0, 128.0, 65536).to(torch.bfloat16).unique()
+    n = (gate.numel() // 8) * 8
+    gate = gate[:n]
+    up = torch.tensor([1.0, -3.5, 0.0078125, 200.0], dtype=torch.bfloat16)
+    y = torch.cat([gate.repeat(4, 1), up[:, None].expand(4, n)], dim=1).contiguous()
+    h = nv.silu_mul(y.cuda())
+    torch.cuda.synchronize()
+    ref = from_bits(orc.silu_mul(bits(y))).float()
+    got = h.float().cpu()
+    ulp = torch.clamp(ref.abs(), min=2.0 ** -126) * 2.0 ** -7
+    bad = (got - ref).abs() > ulp
+    assert not torch.any(bad), (gate.repeat(4, 1)[bad][:5], got[bad][:5], ref[bad][:5])
+
+
 def test_mlp32k_pipeline_full(nv, orc):
     """X 32768x5120 (5 outlier channels x30) -> gate_up W 34816x5120 ->
     silu*mul -> requantize h (dynamic global) -> down W 5120x17408, all on the

@@ -138,3 +138,26 @@ def test_linear_decode_full_size_against_oracle(nv, orc):
     ref = orc.gemm(qx, qw)
     gemm_check(y, ref, norms(orc, qx), norms(orc, qw), "decode 8x17408->5120")
     assert nv.read_fault() == 0
+
+
+def test_linear_reused_workspace_with_stale_padding(nv, orc):
+    """nvfp4_linear leaves the scale bytes of its private quantized X's
+    padding rows unwritten for fewer than 32 tokens (only its GEMM reads them,
+    against zero-filled codes). A workspace that held a 31-token and then a
+    256-token call's data gives a 1-token call the bits of quantize + GEMM,
+    and the oracle's result within the tolerance, for both GEMM kernels'
+    reuse orders."""
+    k, n = 5120, 2048
+    qw = orc.quantize(bits(gaussian(n, k, 9, 0.02)))
+    W = upload(qw)
+    ws = nv.linear_workspace(256, n, k)
+    for m_prev in (31, 256):
+        nv.linear(gaussian(m_prev, k, m_prev).cuda(), W, workspace=ws)
+    x = gaussian(1, k, 4242)
+    y = nv.linear(x.cuda(), W, out_dtype=torch.float32, workspace=ws)
+    y2 = nv.gemm(nv.quantize(x.cuda()), W, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+    qx = orc.quantize(bits(x))
+    gemm_check(y, orc.gemm(qx, qw), norms(orc, qx), norms(orc, qw), "stale padding")
+    assert nv.read_fault() == 0
