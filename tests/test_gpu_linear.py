@@ -150,7 +150,8 @@ def test_linear_reused_workspace_with_stale_padding(nv, orc):
     k, n = 5120, 2048
     qw = orc.quantize(bits(gaussian(n, k, 9, 0.02)))
     W = upload(qw)
-    ws = nv.linear_workspace(256, n, k)
+    nb = max(nv.linear_workspace_bytes(m, n, k) for m in (1, 31, 256))
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
     for m_prev in (31, 256):
         nv.linear(gaussian(m_prev, k, m_prev).cuda(), W, workspace=ws)
     x = gaussian(1, k, 4242)
