@@ -170,13 +170,20 @@ nvfp4_status nvfp4_calibrate_global(const void* x, int64_t rows, int64_t k,
                                     size_t workspace_bytes,
                                     nvfp4_stream_t stream);
 
-/* Workspace bytes nvfp4_gemm can use: for m <= 64, 16*ceil(n/128) bytes of
- * reduction counters (rounded up to 256) plus ceil(n/128)*9*m*128*4 bytes of
- * FP32 partial slabs: with fewer 128-row weight tiles than SMs, few-token
- * GEMMs deal the (tile, k-tile) iterations out to every SM in equal
- * contiguous shares (stream-K) and add the partial tiles in a fixed order;
- * else 0. Passing less (or NULL) is allowed and only disables the
- * stream-K split. */
+/* Workspace bytes nvfp4_gemm can use. It starts with the split GEMMs'
+ * reduction counters: 4 * max(4*ceil(n/128), 64*16) bytes rounded up to 256,
+ * a region that depends on n only. Then:
+ *   m <= 64: ceil(n/128)*9*m*128*4 bytes of FP32 partial slabs. With fewer
+ *     128-row weight tiles than SMs, few-token GEMMs deal the (tile,
+ *     k-tile) iterations out to every SM in equal contiguous shares
+ *     (stream-K) and add the partial tiles in a fixed order.
+ *   m > 64 with at most 64 tiles of 256x256 and k >= 8192: tiles*S*256 KiB
+ *     of FP32 partial tiles, S = min(4, k/4096): when the tiles cannot
+ *     occupy half the CTA pairs, K is cut into up to S slices (split-K, at
+ *     least 16 k-tiles of 256 each) and the last slice of each tile region
+ *     adds the partials in slice order.
+ *   otherwise 0.
+ * Passing less (or NULL) is allowed and only disables the split. */
 size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -199,7 +206,8 @@ size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              (the call zeroes the reduction counters itself).
  * m <= 64 runs the few-token kernel (weights on the MMA's 128-row side,
  * tokens as its N); larger m the paired-CTA 256x256-tile kernel. Results do
- * not depend on the run: partial tiles are summed in k order.
+ * not depend on the run: partial tiles are summed in k order (a workspace
+ * too small for the split gives the unsplit kernel's k order instead).
  * The kernel is launched with programmatic stream serialisation; it reads and
  * writes global memory only after the previous kernel in the stream finished.
  * Errors: INVALID_ARG, MISALIGNED, UNSUPPORTED, CUDA.
@@ -211,9 +219,11 @@ nvfp4_status nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf,
                         int64_t k, void* workspace, size_t workspace_bytes,
                         nvfp4_stream_t stream);
 
-/* Workspace bytes of nvfp4_linear: the quantized activations (codes, scales,
- * global), the amax pass's partial maxima and, for m <= 64, the few-token
- * GEMM's reduction counters and slabs. 0 for invalid sizes. */
+/* Workspace bytes of nvfp4_linear: the split GEMMs' reduction counters (the
+ * n-only region nvfp4_gemm_workspace_bytes starts with, always present) and
+ * their partials where nvfp4_gemm would split, then the quantized
+ * activations (codes, scales, global) and the amax pass's partial maxima.
+ * 0 for invalid sizes. */
 size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
 
 /*
@@ -236,7 +246,13 @@ size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              256-byte aligned, owned by the caller, not shared with a call
  *              that may run at the same time, and zero-filled before its
  *              first use: each call leaves the bytes that must start at zero
- *              zeroed again (after a kernel timeout, zero it again).
+ *              (the counters at its start) zeroed again (after a kernel
+ *              timeout, zero it again). One workspace may serve calls with
+ *              the same n and different m (and k) if it is large enough for
+ *              each: the counters region depends on n only. For fewer than
+ *              32 tokens the
+ *              scales of the quantized X's padding rows are not written
+ *              (only this call's GEMM reads them, against zero codes).
  * Errors: INVALID_ARG (null pointer, bad size, short workspace), MISALIGNED,
  * UNSUPPORTED (k % 32 != 0, sizes >= 2^31), CUDA.
  */

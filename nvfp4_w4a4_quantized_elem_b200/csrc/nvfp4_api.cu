@@ -178,15 +178,26 @@ nvfp4_status launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block,
   return NVFP4_OK;
 }
 
-// Few-token GEMM workspace: reduction counters (4 per 128 weight rows), then
-// kMaxContrib FP32 slabs of [m][128] per weight tile.
-size_t skinny_counter_bytes(int64_t n) {
-  return round_up(static_cast<size_t>(ceil_div(n, 128)) * 4 * sizeof(unsigned int), 256);
+constexpr int64_t kSplitMaxTiles = 64;  // paired split-K: at most this many 256x256 tiles
+
+// The reduction counters of both split GEMMs sit at the start of a GEMM or
+// linear workspace, in a region whose size depends on n only (few-token
+// kernel: 4 per 128 weight rows; paired split-K: 16 per tile, at most
+// kSplitMaxTiles tiles). Every call leaves them zero and nothing else is
+// ever placed there, so one workspace that is large enough for each call
+// may serve calls of different m.
+size_t split_counter_bytes(int64_t n) {
+  int64_t c = ceil_div(n, 128) * 4;
+  if (c < kSplitMaxTiles * 16) c = kSplitMaxTiles * 16;
+  return round_up(static_cast<size_t>(c) * sizeof(unsigned int), 256);
 }
+
+// Few-token GEMM workspace: the counters, then kMaxContrib FP32 slabs of
+// [m][128] per weight tile.
 size_t skinny_workspace_bytes(int64_t m, int64_t n) {
-  return skinny_counter_bytes(n) + static_cast<size_t>(ceil_div(n, 128)) *
-                                       nvfp4::skinny::kMaxContrib * static_cast<size_t>(m) *
-                                       nvfp4::skinny::BW * sizeof(float);
+  return split_counter_bytes(n) + static_cast<size_t>(ceil_div(n, 128)) *
+                                      nvfp4::skinny::kMaxContrib * static_cast<size_t>(m) *
+                                      nvfp4::skinny::BW * sizeof(float);
 }
 
 // Split-K of the paired kernel (nvfp4::gemm, m > 64): when the 256x256 tiles
@@ -196,7 +207,6 @@ size_t skinny_workspace_bytes(int64_t m, int64_t n) {
 // 60 units instead of 20. Workspace: counters (16 per tile), then the FP32
 // partial tiles. The workspace bytes depend on the shape only (the largest
 // S any device could use); the launch picks S from the SM count.
-constexpr int64_t kSplitMaxTiles = 64;
 int64_t paired_tiles(int64_t m, int64_t n) {
   return ceil_div(m, nvfp4::gemm::BM) * ceil_div(n, nvfp4::gemm::BN);
 }
@@ -206,12 +216,10 @@ int paired_split_cap(int64_t m, int64_t n, int64_t k) {
   if (m <= 64 || paired_tiles(m, n) > kSplitMaxTiles || kt < 2 * kMinSliceKTiles) return 1;
   return static_cast<int>(kt / kMinSliceKTiles < kMaxSplitK ? kt / kMinSliceKTiles : kMaxSplitK);
 }
-size_t paired_counter_bytes(int64_t tiles) {
-  return round_up(static_cast<size_t>(tiles) * 16 * sizeof(unsigned int), 256);
-}
-size_t paired_split_bytes(int64_t tiles, int split) {
-  return paired_counter_bytes(tiles) + static_cast<size_t>(tiles) * static_cast<size_t>(split) *
-                                           16 * nvfp4::gemm::kRegionFloats * sizeof(float);
+size_t paired_split_bytes(int64_t m, int64_t n, int split) {
+  return split_counter_bytes(n) + static_cast<size_t>(paired_tiles(m, n)) *
+                                      static_cast<size_t>(split) * 16 *
+                                      nvfp4::gemm::kRegionFloats * sizeof(float);
 }
 int paired_split(int sms, int64_t m, int64_t n, int64_t k) {
   const int cap = paired_split_cap(m, n, k);
@@ -473,7 +481,7 @@ size_t nvfp4_gemm_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   if (m <= 64) return skinny_workspace_bytes(m, n);
   // paired kernel with few tiles: split-K counters and FP32 partial tiles
   const int cap = paired_split_cap(m, n, k);
-  return cap >= 2 ? paired_split_bytes(paired_tiles(m, n), cap) : 0;
+  return cap >= 2 ? paired_split_bytes(m, n, cap) : 0;
 }
 
 }  // extern "C"
@@ -596,9 +604,9 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
       grid = g;
       p.tile_count = static_cast<unsigned int*>(workspace);
       p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                           skinny_counter_bytes(n));
+                                           split_counter_bytes(n));
       if (zero_counters &&
-          cudaMemsetAsync(workspace, 0, skinny_counter_bytes(n), s) != cudaSuccess) {
+          cudaMemsetAsync(workspace, 0, split_counter_bytes(n), s) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
       }
@@ -662,13 +670,13 @@ nvfp4_status gemm_paired(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
   p.split = 1;
   if (p.fused == kPlain && workspace != nullptr && aligned(workspace, 16)) {
     const int sk = paired_split(st->sms, m, n, k);
-    if (sk >= 2 && workspace_bytes >= paired_split_bytes(tiles, sk)) {
+    if (sk >= 2 && workspace_bytes >= paired_split_bytes(m, n, sk)) {
       p.split = sk;
       p.tile_count = static_cast<unsigned int*>(workspace);
       p.partial = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) +
-                                           paired_counter_bytes(tiles));
+                                           split_counter_bytes(n));
       if (zero_counters &&
-          cudaMemsetAsync(workspace, 0, paired_counter_bytes(tiles), stream) != cudaSuccess) {
+          cudaMemsetAsync(workspace, 0, split_counter_bytes(n), stream) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
       }
@@ -771,7 +779,10 @@ nvfp4_status nvfp4_selftest_gemm_stall(const uint8_t* a_codes, const uint8_t* a_
 
 size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k) {
   if (m < 1 || n < 1 || k < 32 || k % 32 != 0) return 0;
-  size_t b = round_up(nvfp4_gemm_workspace_bytes(m, n, k), 256);  // split / stream-K
+  // the split counters' region always (see split_counter_bytes), then the
+  // split GEMMs' partials
+  size_t b = round_up(nvfp4_gemm_workspace_bytes(m, n, k), 256);
+  if (b < split_counter_bytes(n)) b = split_counter_bytes(n);
   b += round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);  // codes
   b += round_up(nvfp4_sf_bytes(m, k), 256);                                // scales
   b += 256;                                                                // global
@@ -803,7 +814,8 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // workspace: [counters + slabs (split work)][codes][scales][global][partials]
   uint8_t* w = static_cast<uint8_t*>(workspace);
-  const size_t split_bytes = round_up(nvfp4_gemm_workspace_bytes(m, n, k), 256);
+  size_t split_bytes = round_up(nvfp4_gemm_workspace_bytes(m, n, k), 256);
+  if (split_bytes < split_counter_bytes(n)) split_bytes = split_counter_bytes(n);
   uint8_t* a_codes = w + split_bytes;
   uint8_t* a_sf = a_codes + round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);
   float* a_global = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(m, k), 256));

@@ -198,7 +198,8 @@ def test_linear_workspace_bytes(L):
     slabs = w_tiles * 9 * m * 128 * 4
     assert f(m, n, k) >= m * k // 2 + L.nvfp4_sf_bytes(m, k) + 16384 + slabs
     assert f(65, n, k) < f(64, n, k)         # no split workspace above 64 tokens
-    assert L.nvfp4_gemm_workspace_bytes(m, n, k) == 256 + slabs
+    # the split counters' region (n only: at least 64 tiles x 16 counters) + slabs
+    assert L.nvfp4_gemm_workspace_bytes(m, n, k) == 4096 + slabs
     assert L.nvfp4_gemm_workspace_bytes(65, n, k) == 0
 
 

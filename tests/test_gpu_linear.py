@@ -29,9 +29,10 @@ def gaussian(rows, k, seed, sigma=1.0):
 
 
 def counter_bytes(n):
-    """Split counters at the start of the few-token workspace: 16 bytes per
-    128 weight rows, rounded up to 256 (nvfp4.h)."""
-    return -(-(16 * -(-n // 128)) // 256) * 256
+    """Split counters at the start of a GEMM / linear workspace (nvfp4.h):
+    4 per 128 weight rows, at least 64 x 16 (the paired kernel's split-K),
+    4 bytes each, rounded up to 256."""
+    return -(-(4 * max(4 * -(-n // 128), 64 * 16)) // 256) * 256
 
 
 @pytest.mark.parametrize("m", [1, 8, 16, 33, 64, 65, 300])
