@@ -157,7 +157,8 @@ def test_linear_reused_workspace_with_stale_padding(nv, orc):
         nv.linear(gaussian(m_prev, k, m_prev).cuda(), W, workspace=ws)
     x = gaussian(1, k, 4242)
     y = nv.linear(x.cuda(), W, out_dtype=torch.float32, workspace=ws)
-    y2 = nv.gemm(nv.quantize(x.cuda()), W, out_dtype=torch.float32)
+    gws = torch.empty(nv.gemm_workspace_bytes(1, n, k), dtype=torch.uint8, device="cuda")
+    y2 = nv.gemm(nv.quantize(x.cuda()), W, out_dtype=torch.float32, workspace=gws)  # same split
     torch.cuda.synchronize()
     assert torch.equal(y, y2)
     qx = orc.quantize(bits(x))
