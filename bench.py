@@ -444,18 +444,81 @@ def timed(stream, fn, reps, flush=None, tag=1):
     return statistics.mean(a.elapsed_time(b) for a, b in evs)
 
 
-def quantizer_alone(nv, x, stream, flush, reps=10):
+def quantizer_alone(nv, x, stream, flush=None, reps=10):
     """The quantizer kernel alone (static global: no amax pass) over x into
-    a scratch output, L2 flushed before each call: GB/s of its 2.5625 B per
-    element."""
+    a scratch output: GB/s of its 2.5625 B per element. Calls run back to
+    back in one CUDA graph, each on its own copy of x (R copies totalling
+    at least 2x L2, so every call streams its x from HBM), the graph
+    replayed and timed as a whole: the kernel's throughput without the
+    launch and event cost of a lone call."""
     g = torch.full((1,), 7.0, dtype=torch.float32, device=x.device)
-    out = nv.NVFP4Tensor.empty(x.shape[0], x.shape[1], x.device)
-    ms = timed(stream, lambda: nv.quantize(x, global_scale=g, out=out, stream=stream), reps,
-               flush, 3)
+    nbytes = x.shape[0] * x.shape[1] * 2
+    R = max(1, math.ceil(2 * L2_BYTES / nbytes))
+    xs = [x] + [x.clone() for _ in range(R - 1)]
+    outs = [nv.NVFP4Tensor.empty(x.shape[0], x.shape[1], x.device) for _ in range(R)]
+
+    def calls():
+        for xi, oi in zip(xs, outs):
+            nv.quantize(xi, global_scale=g, out=oi, stream=stream)
+
+    with torch.cuda.stream(stream):
+        calls()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        calls()
+    n = max(2, math.ceil(reps / R))
+    with torch.cuda.stream(stream):
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            graph.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / (n * R)
+    del graph, xs, outs
     elems = x.shape[0] * x.shape[1]
-    del out
     return {"shape": list(x.shape), "ms": round(ms, 5),
-            "gbs": round(elems * QUANT_BYTES_PER_ELEM / (ms * 1e-3) / 1e9, 1)}
+            "gbs": round(elems * QUANT_BYTES_PER_ELEM / (ms * 1e-3) / 1e9, 1),
+            "timing": f"{n} replays of a graph of {R} calls on {R} copies of x"}
+
+
+def gemm_alone(nv, A, B, y, ws, stream, reps=12):
+    """The GEMM kernel alone on the step's operands: back-to-back calls in one
+    CUDA graph, each on its own copy of A and of Y (R copies, so that each
+    call's A and Y total at least 2x L2 over the rotation), the graph
+    replayed and timed as a whole: the kernel's duration without the launch
+    and event cost of a lone call. Returns (ms per call, description)."""
+    per_call = A.codes.numel() + A.sf.numel() + y.numel() * y.element_size()
+    R = max(1, math.ceil(2 * L2_BYTES / per_call))
+    As = [A] + [nv.NVFP4Tensor(A.codes.clone(), A.sf.clone(), A.global_scale.clone(), A.rows, A.k)
+                for _ in range(R - 1)]
+    ys = [y] + [torch.empty_like(y) for _ in range(R - 1)]
+
+    def calls():
+        for a, yy in zip(As, ys):
+            nv.gemm(a, B, out=yy, workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        calls()
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        calls()
+    n = max(2, math.ceil(reps / R))
+    with torch.cuda.stream(stream):
+        graph.replay()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n):
+            graph.replay()
+        e1.record(stream)
+    stream.synchronize()
+    ms = e0.elapsed_time(e1) / (n * R)
+    del graph, As, ys
+    return ms, (f"{n} replays of a CUDA graph of {R} GEMM calls, each on its own copy of A and "
+                "Y, one event pair around all")
 
 
 def cublaslt_reference(A, B, stream, flush, reps=10):
@@ -539,15 +602,14 @@ def prefill_components(wk, step, stream, flush, phase_ms, pk):
     if step.kind == "linear":
         qd = timed(s, lambda: nv.quantize(wk["x"], global_scale=wk.get("x_global"), out=step.A,
                                           workspace=step.ws, stream=s), 10, flush, 5)
-        g_ms = timed(s, lambda: nv.gemm(step.A, wk["W"], out=step.y, workspace=step.gws,
-                                        stream=s), 10, flush, 5)
+        g_ms, g_how = gemm_alone(nv, step.A, wk["W"], step.y, step.gws, s)
         (mm, nn, kk) = wk["gemms"][0]
         lib = cublaslt_reference(step.A, wk["W"], s, flush) if mm > 64 else None
-        comp["phase_timing"] = ("quantizer (as in the step) and GEMM each launched alone, 10 "
-                                "times, CUDA events on their stream, L2 flushed before each")
+        comp["phase_timing"] = ("quantizer (as in the step) launched alone 10 times, CUDA "
+                                "events on its stream, L2 flushed before each; GEMM: " + g_how)
         comp["quantize_ms"] = round(qd, 5)
         comp["gemm_ms"] = round(g_ms, 5)
-        comp["quant"] = quantizer_alone(nv, wk["x"], s, flush)
+        comp["quant"] = quantizer_alone(nv, wk["x"], s)
         roof = tensor_roofline(name, 2 * mm * nn * kk, g_ms, pk,
                                "nvfp4::gemm::gemm_kernel" if mm > 64 else
                                "nvfp4::skinny::skinny_kernel", lib)
@@ -555,14 +617,14 @@ def prefill_components(wk, step, stream, flush, phase_ms, pk):
     (m1, n1, k1), (m2, n2, k2) = wk["gemms"]
     f1, f2 = 2 * m1 * n1 * k1, 2 * m2 * n2 * k2
     comp["phase_ms"] = [round(v, 5) for v in phase_ms]
-    comp["quant_x"] = quantizer_alone(nv, wk["x"], s, flush)
+    comp["quant_x"] = quantizer_alone(nv, wk["x"], s)
     down_ms = timed(s, lambda: nv.gemm(step.H, wk["Wd"], out=step.y, stream=s), 5, flush, 5)
     comp["down_gemm"] = {"ms": round(down_ms, 5), "tflops": round(f2 / (down_ms * 1e-3) / 1e12, 1)}
     if step.kind == "mlp":
         call_ms = timed(s, lambda: nv.gemm_swiglu_quant_dynamic(step.A, wk["Wgi"], out=step.H,
                                                                 workspace=step.hws, stream=s),
                         5, flush, 5)
-        comp["quant_h"] = quantizer_alone(nv, step.h_bf16(), s, flush, reps=5)
+        comp["quant_h"] = quantizer_alone(nv, step.h_bf16(), s, reps=5)
         g_ms = call_ms - comp["quant_h"]["ms"]
         comp["gate_up_call_ms"] = round(call_ms, 5)
         comp["phase_timing"] = (
@@ -580,7 +642,7 @@ def prefill_components(wk, step, stream, flush, phase_ms, pk):
         lib = cublaslt_reference(step.A, wk["Wgi"], s, flush, reps=5)
     else:
         g_ms = timed(s, lambda: nv.gemm(step.A, wk["Wgu"], out=step.ygu, stream=s), 5, flush, 5)
-        comp["quant_h"] = quantizer_alone(nv, step.h, s, flush, reps=5)
+        comp["quant_h"] = quantizer_alone(nv, step.h, s, reps=5)
         comp["phase_timing"] = "each call alone, 5 times, L2 flushed before each"
         kernel = "nvfp4::gemm::gemm_kernel (gate_up, bf16 out)"
         lib = cublaslt_reference(step.A, wk["Wgu"], s, flush, reps=5)
