@@ -301,15 +301,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
       // The first ring's worth of stages needs no empty-slot wait. With
       // early_w their weight halves are requested before the grid-dependency
       // wait, the token halves after it.
+      // Every weight byte is read once per call: its lines leave L2 first.
+      const uint64_t wpol = ptx::l2_policy_evict_first();
       int npre = 0;
       if (p.early_w) {
         WorkIter w = it;
         for (; npre < C::STAGES && w.sg.valid; ++npre, w.next(p)) {
           uint8_t* st = smem + npre * C::STAGE_BYTES;
           ptx::mbar_arrive_expect_tx(&full[npre], C::STAGE_RAW);
-          ptx::tma_load_2d(st, &tmW, &full[npre], w.kt * BK_BYTES, w.sg.wt * BW);
-          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4,
-                           w.sg.wt);
+          ptx::tma_load_2d_hint(st, &tmW, &full[npre], w.kt * BK_BYTES, w.sg.wt * BW, wpol);
+          ptx::tma_load_3d_hint(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4,
+                                w.sg.wt, wpol);
+        }
+        // The rest of this CTA's weights go to L2 right away: while this
+        // kernel waits for its predecessors (in a decode step, the previous
+        // layer's GEMM and this layer's quantizer) HBM keeps streaming the
+        // weights, and the ring refills from L2 once the MMAs start.
+        for (; w.sg.valid; w.next(p)) {
+          ptx::tma_prefetch_l2_2d(&tmW, w.kt * BK_BYTES, w.sg.wt * BW);
+          ptx::tma_prefetch_l2_3d(&tmSFW, 0, w.kt * 4, w.sg.wt);
         }
       }
       ptx::grid_dep_wait();
@@ -338,10 +348,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
         }
         uint8_t* st = smem + stage * C::STAGE_BYTES;
         ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
-        ptx::tma_load_2d(st, &tmW, &full[stage], it.kt * BK_BYTES, it.sg.wt * BW);
+        ptx::tma_load_2d_hint(st, &tmW, &full[stage], it.kt * BK_BYTES, it.sg.wt * BW, wpol);
         ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], it.kt * BK_BYTES, 0);
-        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, it.kt * 4,
-                         it.sg.wt);
+        ptx::tma_load_3d_hint(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, it.kt * 4,
+                              it.sg.wt, wpol);
         ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
                          it.kt * 4, 0);
         pending |= 1u << stage;
