@@ -313,14 +313,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 2)
           ptx::tma_load_3d_hint(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4,
                                 w.sg.wt, wpol);
         }
-        // The rest of this CTA's weights go to L2 right away: while this
-        // kernel waits for its predecessors (in a decode step, the previous
-        // layer's GEMM and this layer's quantizer) HBM keeps streaming the
-        // weights, and the ring refills from L2 once the MMAs start.
-        for (; w.sg.valid; w.next(p)) {
-          ptx::tma_prefetch_l2_2d(&tmW, w.kt * BK_BYTES, w.sg.wt * BW);
-          ptx::tma_prefetch_l2_3d(&tmSFW, 0, w.kt * 4, w.sg.wt);
-        }
       }
       ptx::grid_dep_wait();
       for (int i = 0; i < npre; ++i, it.next(p)) {

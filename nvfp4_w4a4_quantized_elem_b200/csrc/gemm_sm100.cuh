@@ -495,21 +495,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // halves are requested before the grid-dependency wait.
       int npre = 0;
       if (p.early_w) {
-        Item w = it;
-        for (; npre < STAGES && w.t < num_units; ++npre, w = next(w)) {
+        for (Item w = it; npre < STAGES && w.t < num_units; ++npre, w = next(w)) {
           if (leader) ptx::mbar_arrive_expect_tx(&full[npre], 2 * STAGE_BYTES);
           load_b(w, static_cast<uint32_t>(npre));
-        }
-        // One work unit per pair (a decode step's GEMM): the rest of this
-        // unit's B goes to L2 now, so HBM keeps streaming the weights while
-        // the kernel waits for its predecessor; the ring then refills from
-        // L2. (With several units per pair B is shared through L2 anyway.)
-        if (num_units <= num_pairs) {
-          for (; w.t == pair; w = next(w)) {
-            ptx::tma_prefetch_l2_2d(&tmB, w.kt * BK_BYTES,
-                                    w.nb * BN + static_cast<int>(rank) * HALF);
-            ptx::tma_prefetch_l2_3d(&tmSFB, 0, w.kt * 4, w.nb * 2);
-          }
         }
       }
       ptx::grid_dep_wait();

@@ -146,22 +146,6 @@ __device__ __forceinline__ void tma_load_3d_hint(void* dst, const void* tmap, ui
       : "memory");
 }
 
-// Bring a tile into L2 only (no shared memory, no completion signal).
-__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(x), "r"(y)
-               : "memory");
-}
-
-__device__ __forceinline__ void tma_prefetch_l2_3d(const void* tmap, int32_t x, int32_t y,
-                                                   int32_t z) {
-  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global [%0, {%1, %2, %3}];" ::"l"(
-                   reinterpret_cast<uint64_t>(tmap)),
-               "r"(x), "r"(y), "r"(z)
-               : "memory");
-}
-
 // L2 policy: lines the holder reads once leave L2 first.
 __device__ __forceinline__ uint64_t l2_policy_evict_first() {
   uint64_t pol;
