@@ -58,16 +58,18 @@ constexpr int BK_BYTES = BK / 2;
 constexpr int NUM_THREADS = 256;
 constexpr int SF_WARP0 = 2;       // warps 2, 3 copy scales
 constexpr int EPI_WARP0 = 4;      // warps 4..7 drain the accumulator
-// Half of an SM per CTA (tensor memory, shared memory, registers), so that
-// a CTA of the next decode layer's GEMM can start on the same SM while this
-// one drains: its first weight tiles then stream during this one's tail.
-constexpr uint32_t TMEM_COLS = 256;
+// One CTA per SM with the deepest ring that fits: in a decode layer
+// sequence the ring's first stages are requested before the grid-dependency
+// wait, and the deeper the ring the more of the weight stream overlaps the
+// wait for the previous layer and this layer's quantizer (measured on a
+// graph of 8 decode steps: 8 stages beat a half-SM CTA with 5 stages that
+// let the next layer's CTA start beside it, by 0.3-1.2 us per step).
+constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_BUF_COLS = 32;  // per scale buffer: weights 16, tokens 16
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 100000000ull;
-// dynamic shared memory per CTA such that two CTAs fit in an SM's 228 KiB
-// (each CTA also holds 1 KiB reserved by the system)
-constexpr size_t kSmemPerCta = 114 * 1024;
+// dynamic shared memory per CTA (of the 227 KiB a CTA may use)
+constexpr size_t kSmemPerCta = 220 * 1024;
 constexpr int kMaxSplits = 8;     // stream-K: at most this many CTAs per weight tile
 constexpr int kMaxContrib = kMaxSplits + 1;  // contributor slots per tile (host-checked)
 constexpr int kSumTokens = 8;     // tokens summed per round of slab loads
@@ -87,7 +89,7 @@ struct Cfg {
   static constexpr int STAGES_FIT = static_cast<int>((kSmemPerCta - 1024 - 512) / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
   static constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
-  static_assert(SMEM_BYTES <= kSmemPerCta, "two CTAs per SM");
+  static_assert(SMEM_BYTES <= kSmemPerCta, "shared memory per CTA");
   // two BNT-column accumulators (a segment's MMAs run while the epilogue
   // drains the previous segment), then one scale buffer per stage
   static constexpr int NSF = STAGES;
@@ -236,7 +238,7 @@ __device__ __forceinline__ void sum_slabs(const float* col, int64_t slab, int m0
 }
 
 template <int BNT>
-__global__ void __launch_bounds__(NUM_THREADS, 2)
+__global__ void __launch_bounds__(NUM_THREADS, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                   const __grid_constant__ CUtensorMap tmSFW,
                   const __grid_constant__ CUtensorMap tmSFX, const Params p) {
