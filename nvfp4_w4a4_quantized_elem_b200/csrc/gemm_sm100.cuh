@@ -179,10 +179,9 @@ constexpr int kMinSliceKTiles = 16;      // k-tiles per slice at least (host-che
 // one operand (M-tiles when !raster_n, N-tiles when raster_n) and then step
 // along the other, so the pairs resident at one time share operand tiles in
 // L2 and the band's rows of its operand stay in L2 while the other operand
-// streams past once per band. The host sizes the band so that it fits in
-// L2: a whole operand of at most ~48 MB is kept resident (the other read
-// once), else the band is cut to ~48 MB of A. (Fixed 16-tile bands re-read
-// the 89 MB gate_up weight 8 times and the down projection's A 3 times.)
+// streams past once per band. The host sizes the band (about 24 MB of the
+// banded operand) and picks the direction with the smaller DRAM read
+// traffic. (Fixed 16-tile M bands re-read the 89 MB gate_up weight 8 times.)
 __device__ __forceinline__ void tile_coords(int t, const Params& p, int& mb, int& nb) {
   const int nb_band = p.raster_n ? p.num_n_blk : p.num_m_blk;  // tiles along the band's side
   const int nb_walk = p.raster_n ? p.num_m_blk : p.num_n_blk;
