@@ -232,9 +232,13 @@ size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * 4-bit tensor cores): Y = dequant(quantize(X)) @ dequant(W)^T, i.e.
  * nvfp4_quantize of X into the workspace followed by nvfp4_gemm, with
  * identical results. The GEMM is launched to start while the quantizer runs:
- * its set-up and its first weight tiles overlap the quantization. This
- * relies on W, w_sf and w_global being written before the call (by work
- * already in the stream or earlier), never by a kernel launched in between.
+ * its set-up and its first weight tiles overlap the quantization. For at
+ * most 8 tokens there is no quantizer kernel: the few-token GEMM quantizes
+ * each k-tile of X as it lands in shared memory (same arithmetic, same
+ * bits), after an amax pass only when the global is dynamic and X exceeds
+ * NVFP4_ONE_PASS_MAX_BYTES. This relies on W, w_sf and w_global being
+ * written before the call (by work already in the stream or earlier), never
+ * by a kernel launched in between.
  *   x         device bf16 [m][ldx], 16-byte aligned, ldx >= k, ldx % 8 == 0.
  *   x_global  NULL: dynamic global scale of X (amax pass, or none for X of at
  *             most NVFP4_ONE_PASS_MAX_BYTES, as in nvfp4_quantize); else a
@@ -249,10 +253,10 @@ size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  *              (the counters at its start) zeroed again (after a kernel
  *              timeout, zero it again). One workspace may serve calls with
  *              the same n and different m (and k) if it is large enough for
- *              each: the counters region depends on n only. For fewer than
- *              32 tokens the
- *              scales of the quantized X's padding rows are not written
- *              (only this call's GEMM reads them, against zero codes).
+ *              each: the counters region depends on n only. For 9 to 31
+ *              tokens the scales of the quantized X's padding rows are not
+ *              written (only this call's GEMM reads them, against zero
+ *              codes); for at most 8 the quantized X is not stored at all.
  * Errors: INVALID_ARG (null pointer, bad size, short workspace), MISALIGNED,
  * UNSUPPORTED (k % 32 != 0, sizes >= 2^31), CUDA.
  */

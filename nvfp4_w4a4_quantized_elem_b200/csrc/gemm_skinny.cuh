@@ -47,6 +47,7 @@
 
 #include "fault.cuh"
 #include "ptx.cuh"
+#include "quant.cuh"
 
 namespace nvfp4 {
 
@@ -55,9 +56,10 @@ namespace skinny {
 constexpr int BW = 128;           // weight rows per tile (MMA M)
 constexpr int BK = 256;           // FP4 elements per k-tile
 constexpr int BK_BYTES = BK / 2;
-constexpr int NUM_THREADS = 256;
 constexpr int SF_WARP0 = 2;       // warps 2, 3 copy scales
 constexpr int EPI_WARP0 = 4;      // warps 4..7 drain the accumulator
+constexpr int XQ_WARP0 = 8;       // warps 8..11 quantize the tokens (in-kernel mode)
+constexpr int XQ_THREADS = 128;
 // One CTA per SM with the deepest ring that fits: in a decode layer
 // sequence the ring's first stages are requested before the grid-dependency
 // wait, and the deeper the ring the more of the weight stream overlaps the
@@ -76,19 +78,40 @@ constexpr int kSumTokens = 8;     // tokens summed per round of slab loads
 
 enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, kFaultScales = 128u };
 
-template <int BNT>
+constexpr int XR = 8;             // in-kernel mode: bf16 token rows per stage (m <= XR)
+// in-kernel mode, dynamic global: X of at most quant::kSelfAmaxBytes (64 KiB)
+// takes its max inside the kernel, in one round of loads by warps 4..11
+// (larger X comes with the amax pass's partial maxima: a second round, 148
+// CTAs each reading all of X, measured slower than the amax pass)
+constexpr int XMAX_THREADS = 256;
+
+// FUSED: the tokens (m <= XR) arrive in bf16 (one [XR][256] tile per stage, by
+// TMA with the weights) and warps 8..11 quantize them into the stage, in the
+// code and scale layouts the TMA would have written (see skinny_kernel).
+template <int BNT, bool FUSED>
 struct Cfg {
   static_assert(BNT == 16 || BNT == 32 || BNT == 64, "token tile (few-token kernel: m <= 64)");
+  static_assert(!FUSED || BNT == 16, "in-kernel token quantization: m <= XR, one 16-token tile");
+  static constexpr int THREADS = FUSED ? 32 * XQ_WARP0 + XQ_THREADS : 32 * XQ_WARP0;
   static constexpr int A_BYTES = BW * BK_BYTES;             // 16 KiB of weights
   static constexpr int B_BYTES = (BNT < 8 ? 8 : BNT) * BK_BYTES;
   static constexpr int SFB_BLOCKS = (BNT + 127) / 128;      // 128-row scale blocks of tokens
   static constexpr int SFA_BYTES = 2048;
   static constexpr int SFB_BYTES = 2048 * SFB_BLOCKS;
-  static constexpr int STAGE_RAW = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int XRAW_OFF = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+  static constexpr int XRAW_BYTES = FUSED ? XR * BK * 2 : 0;  // bf16 tokens of one k-tile
+  static constexpr int STAGE_RAW = XRAW_OFF + XRAW_BYTES;
+  // bytes the TMA brings into a stage
+  static constexpr int TMA_BYTES = FUSED ? A_BYTES + SFA_BYTES + XRAW_BYTES : STAGE_RAW;
   static constexpr int STAGE_BYTES = (STAGE_RAW + 1023) / 1024 * 1024;
-  static constexpr int STAGES_FIT = static_cast<int>((kSmemPerCta - 1024 - 512) / STAGE_BYTES);
+  // after the ring: barriers, then (FUSED) X's global, warp maxima and its
+  // 128-entry table of g / dec(s)
+  static constexpr int TAIL_BYTES = 1536;
+  static constexpr int STAGES_FIT =
+      static_cast<int>((kSmemPerCta - 1024 - TAIL_BYTES) / STAGE_BYTES);
   static constexpr int STAGES = STAGES_FIT > 8 ? 8 : STAGES_FIT;
-  static constexpr size_t SMEM_BYTES = 1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + 512;
+  static constexpr size_t SMEM_BYTES =
+      1024 + static_cast<size_t>(STAGES) * STAGE_BYTES + TAIL_BYTES;
   static_assert(SMEM_BYTES <= kSmemPerCta, "shared memory per CTA");
   // two BNT-column accumulators (a segment's MMAs run while the epilogue
   // drains the previous segment), then one scale buffer per stage
@@ -119,6 +142,16 @@ struct Params {
   // never completes and every role's bounded wait runs into its limit.
   int stall_first_stage;
   uint64_t wait_limit_ns;   // per-wait limit; 0 = kWaitLimitNs
+  // FUSED only: X's global scale, in the order nvfp4_quantize takes it: the
+  // static global x_global_in; else 2688 / max|X| over the amax pass's
+  // x_nparts partial maxima; else (x_nparts == 0) over X itself, which the
+  // host bounds to kSelfAmaxBytes. CTA 0 writes it to x_global_out if set.
+  const uint16_t* x;        // bf16 [M][ldx] (read for the max; tiles come by TMA)
+  int64_t ldx;
+  const float* x_global_in;
+  const float* x_partials;
+  int x_nparts;
+  float* x_global_out;
 };
 
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity,
@@ -153,6 +186,30 @@ __device__ __forceinline__ void tc_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[3
         "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
       : "r"(taddr)
       : "memory");
+}
+
+// FP32 bits of max|x| over the 16-byte chunks i = part, part + nparts, ... of
+// the bf16 X [M][ldx] (row length K): rounds of 16 predicated loads per thread.
+__device__ __forceinline__ uint32_t x_max_part(const uint16_t* x, int64_t ldx, int M, int K,
+                                               uint32_t part, uint32_t nparts) {
+  const uint32_t chunks = static_cast<uint32_t>(K >> 3);
+  const uint32_t total = static_cast<uint32_t>(M) * chunks;
+  uint32_t m = 0;
+  for (uint32_t i = part; i < total; i += 16u * nparts) {
+    uint4 v[16];
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+      const uint32_t e = i + static_cast<uint32_t>(u) * nparts;
+      const uint32_t r = e / chunks;
+      const uint32_t c = e - r * chunks;
+      v[u] = e < total ? __ldg(reinterpret_cast<const uint4*>(
+                             x + static_cast<uint64_t>(r) * static_cast<uint64_t>(ldx) + c * 8u))
+                       : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 16; ++u) m = max(m, quant::absmax_bits8(v[u]) << 16);
+  }
+  return m;
 }
 
 // The CTA that owns stream-K iteration `it` (shares are [c T / G, (c+1) T / G)).
@@ -237,12 +294,12 @@ __device__ __forceinline__ void sum_slabs(const float* col, int64_t slab, int m0
   }
 }
 
-template <int BNT>
-__global__ void __launch_bounds__(NUM_THREADS, 1)
+template <int BNT, bool FUSED>
+__global__ void __launch_bounds__(Cfg<BNT, FUSED>::THREADS, 1)
     skinny_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX,
                   const __grid_constant__ CUtensorMap tmSFW,
                   const __grid_constant__ CUtensorMap tmSFX, const Params p) {
-  using C = Cfg<BNT>;
+  using C = Cfg<BNT, FUSED>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -253,8 +310,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* drain = tmem_empty + 2;
   uint64_t* sf_full = drain + 1;
   uint64_t* drain_sf = sf_full + C::NSF;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
+  uint64_t* xready = drain_sf + 1;           // FUSED: [STAGES] tokens quantized into the stage
+  uint64_t* g_ready = xready + C::STAGES;    // FUSED: X's global and its table are ready
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(g_ready + 1);
   volatile uint32_t* abort_flag = tmem_holder + 1;
+  float* s_gx = reinterpret_cast<float*>(tmem_holder + 2);      // FUSED: X's global
+  uint32_t* s_red = tmem_holder + 8;                            // FUSED: [8] warp maxima
+  float* s_rtab = reinterpret_cast<float*>(tmem_holder + 16);  // FUSED: [128] g / dec(s)
+  // FUSED with a dynamic global and no amax partials: warps 4..11 take
+  // max|X| together, meeting at named barrier 3
+  const bool x_self_max = FUSED && p.x_global_in == nullptr && p.x_nparts == 0;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -273,12 +338,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::mbar_init(&sf_full[b], 2);
     }
     ptx::mbar_init(drain_sf, 2);
+    if (FUSED) {
+      for (int s = 0; s < C::STAGES; ++s) ptx::mbar_init(&xready[s], 1);
+      ptx::mbar_init(g_ready, 1);
+    }
     *abort_flag = 0u;
     ptx::fence_mbarrier_init();
     ptx::tma_prefetch_desc(&tmW);
     ptx::tma_prefetch_desc(&tmX);
     ptx::tma_prefetch_desc(&tmSFW);
-    ptx::tma_prefetch_desc(&tmSFX);
+    if (!FUSED) ptx::tma_prefetch_desc(&tmSFX);
   }
   if (warp == 1) {
     ptx::tmem_alloc(tmem_holder, TMEM_COLS);
@@ -310,7 +379,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         WorkIter w = it;
         for (; npre < C::STAGES && w.sg.valid; ++npre, w.next(p)) {
           uint8_t* st = smem + npre * C::STAGE_BYTES;
-          ptx::mbar_arrive_expect_tx(&full[npre], C::STAGE_RAW);
+          ptx::mbar_arrive_expect_tx(&full[npre], C::TMA_BYTES);
           ptx::tma_load_2d_hint(st, &tmW, &full[npre], w.kt * BK_BYTES, w.sg.wt * BW, wpol);
           ptx::tma_load_3d_hint(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[npre], 0, w.kt * 4,
                                 w.sg.wt, wpol);
@@ -319,9 +388,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       ptx::grid_dep_wait();
       for (int i = 0; i < npre; ++i, it.next(p)) {
         uint8_t* st = smem + i * C::STAGE_BYTES;
-        ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[i], it.kt * BK_BYTES, 0);
-        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[i], 0,
-                         it.kt * 4, 0);
+        if (FUSED) {
+          ptx::tma_load_2d(st + C::XRAW_OFF, &tmX, &full[i], it.kt * BK, 0);
+        } else {
+          ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[i], it.kt * BK_BYTES, 0);
+          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[i], 0,
+                           it.kt * 4, 0);
+        }
         pending |= 1u << i;
       }
       stage = static_cast<uint32_t>(npre % C::STAGES);
@@ -341,13 +414,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           continue;
         }
         uint8_t* st = smem + stage * C::STAGE_BYTES;
-        ptx::mbar_arrive_expect_tx(&full[stage], C::STAGE_RAW);
+        ptx::mbar_arrive_expect_tx(&full[stage], C::TMA_BYTES);
         ptx::tma_load_2d_hint(st, &tmW, &full[stage], it.kt * BK_BYTES, it.sg.wt * BW, wpol);
-        ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], it.kt * BK_BYTES, 0);
         ptx::tma_load_3d_hint(st + C::A_BYTES + C::B_BYTES, &tmSFW, &full[stage], 0, it.kt * 4,
                               it.sg.wt, wpol);
-        ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
-                         it.kt * 4, 0);
+        if (FUSED) {
+          ptx::tma_load_2d(st + C::XRAW_OFF, &tmX, &full[stage], it.kt * BK, 0);
+        } else {
+          ptx::tma_load_2d(st + C::A_BYTES, &tmX, &full[stage], it.kt * BK_BYTES, 0);
+          ptx::tma_load_3d(st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES, &tmSFX, &full[stage], 0,
+                           it.kt * 4, 0);
+        }
         pending |= 1u << stage;
         pending_parity = (pending_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == C::STAGES) {
@@ -379,7 +456,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         ptx::tc_fence_after();
         const uint32_t dacc = tmem + buf * static_cast<uint32_t>(BNT);
         for (int kt = k0; kt < k1; ++kt) {
-          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultMma, lim) ||
+          // FUSED: the quantized tokens are in the stage once xready is
+          // (the token quantizer waited for the stage's TMA data first)
+          if (!wait_bounded(FUSED ? &xready[stage] : &full[stage], phase, abort_flag, kFaultMma,
+                            lim) ||
               !wait_bounded(&sf_full[stage], phase, abort_flag, kFaultMma, lim)) {
             aborted = true;
             break;
@@ -423,8 +503,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (sg.first(p); sg.valid && !aborted; sg.next(p)) {
         for (int kt = sg.k0; kt < sg.k1; ++kt) {
           // the stage's data having landed means its previous MMAs finished
-          // (the producer waited for them), so scale buffer `stage` is free
-          if (!wait_bounded(&full[stage], phase, abort_flag, kFaultScales, lim)) {
+          // (the producer waited for them), so scale buffer `stage` is free;
+          // FUSED: the token scales are in the stage once xready is
+          if (!wait_bounded(FUSED ? &xready[stage] : &full[stage], phase, abort_flag,
+                            kFaultScales, lim)) {
             aborted = true;
             break;
           }
@@ -456,15 +538,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         drain_wait(drain_sf, 0);
       }
     }
-  } else {
+  } else if (warp < XQ_WARP0) {
     // -------------------------------------------------------------- epilogue --
     ptx::grid_dep_wait();  // the globals come from earlier kernels; Y may be in use
+    if (x_self_max) {  // this warp's share of max|X| (chunks 128.., the quantizer warps 0..)
+      uint32_t m = x_max_part(p.x, p.ldx, p.M, p.K,
+                              static_cast<uint32_t>(threadIdx.x - EPI_WARP0 * 32 + XQ_THREADS),
+                              XMAX_THREADS);
+      m = __reduce_max_sync(0xFFFFFFFFu, m);
+      if (lane == 0) s_red[4 + warp - EPI_WARP0] = m;
+      asm volatile("bar.sync 3, %0;" ::"n"(XMAX_THREADS) : "memory");
+    }
     const int q = warp & 3;  // tensor-memory lane quarter (warps 4..7 -> 0..3)
-    const float alpha = 1.0f / (__ldg(p.a_global) * __ldg(p.b_global));
+    bool epi_ok = true;
+    float gx;
+    if (FUSED) {  // X's global, as the token quantizer warps derived it
+      // warp-uniform outcome of every wait: the lanes that saw the phase and
+      // a lane that saw another role's abort must not part ways before the
+      // warp-wide tensor-memory loads
+      epi_ok = __all_sync(0xFFFFFFFFu, wait_bounded(g_ready, 0u, abort_flag, kFaultEpilogue, lim));
+      gx = *s_gx;
+    } else {
+      gx = __ldg(p.a_global);
+    }
+    const float alpha = 1.0f / (gx * __ldg(p.b_global));
     uint32_t acc_phase = 0, buf = 0;  // acc_phase: bit per accumulator
     const int64_t T = static_cast<int64_t>(p.num_w_tiles) * p.num_k_tiles;
     SegIter sg;
-    for (sg.first(p); sg.valid; sg.next(p)) {
+    for (sg.first(p); sg.valid && epi_ok; sg.next(p)) {
       const int wt = sg.wt;
       const bool whole = sg.k0 == 0 && sg.k1 == p.num_k_tiles;  // no other contributor
       int c_first = 0, n_contrib = 1;
@@ -473,7 +574,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         n_contrib = cta_of(static_cast<int64_t>(wt + 1) * p.num_k_tiles - 1, T, gridDim.x) -
                     c_first + 1;
       }
-      if (!wait_bounded(&tmem_full[buf], (acc_phase >> buf) & 1u, abort_flag, kFaultEpilogue, lim))
+      if (!__all_sync(0xFFFFFFFFu, wait_bounded(&tmem_full[buf], (acc_phase >> buf) & 1u,
+                                                abort_flag, kFaultEpilogue, lim)))
         break;
       ptx::tc_fence_after();
       const int nl = q * 32 + lane;            // column within the weight tile
@@ -556,6 +658,131 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           if (lane == 0) p.tile_count[wt * 4 + q] = 0u;  // ready for the next call
         }
+      }
+    }
+  } else if (FUSED) {
+    // ------------------------------------------------------ token quantizer --
+    // nvfp4_quantize's arithmetic on the bf16 token tile each stage receives,
+    // written into the stage in the layouts the TMA would have delivered:
+    // codes as the 128-byte-swizzled K-major B operand, scales as the stage's
+    // four 512-byte atoms. Bit for bit the tokens nvfp4_quantize would write.
+    const int t = threadIdx.x - XQ_WARP0 * 32;  // 0..127
+    auto xq_sync = [] { asm volatile("bar.sync 2, %0;" ::"n"(XQ_THREADS) : "memory"); };
+    // named barrier 2 that also returns whether every thread's predicate held
+    auto xq_sync_and = [](bool pred) {
+      uint32_t all;
+      asm volatile(
+          "{\n\t.reg .pred p, q;\n\t"
+          "setp.ne.u32 p, %1, 0;\n\t"
+          "barrier.cta.red.and.pred q, 2, %2, p;\n\t"
+          "selp.u32 %0, 1, 0, q;\n\t}"
+          : "=r"(all)
+          : "r"(static_cast<uint32_t>(pred)), "n"(XQ_THREADS)
+          : "memory");
+      return all != 0u;
+    };
+    // token codes and scales of every stage start at zero (rows >= M stay
+    // so); no global memory involved, so this overlaps the previous kernel
+    for (int s = 0; s < C::STAGES; ++s) {
+      uint4* zc = reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES + C::A_BYTES);
+      for (int i = t; i < C::B_BYTES / 16; i += XQ_THREADS) zc[i] = make_uint4(0u, 0u, 0u, 0u);
+      uint4* zs = reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES + C::A_BYTES + C::B_BYTES +
+                                           C::SFA_BYTES);
+      for (int i = t; i < C::SFB_BYTES / 16; i += XQ_THREADS) zs[i] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    ptx::grid_dep_wait();  // X, its static global or the amax partials come from earlier kernels
+    if (p.x_global_in != nullptr) {
+      if (t == 0) *s_gx = __ldg(p.x_global_in);
+    } else {
+      uint32_t m = 0;  // FP32 bits of max|X| (non-negative: the bits order as the values)
+      int nwarps = 4;
+      if (p.x_nparts > 0) {
+        for (int i = t; i < p.x_nparts; i += XQ_THREADS)
+          m = max(m, __float_as_uint(__ldcg(p.x_partials + i)));
+      } else {  // X of at most kSelfAmaxBytes, shared with the epilogue warps
+        m = x_max_part(p.x, p.ldx, p.M, p.K, static_cast<uint32_t>(t), XMAX_THREADS);
+        nwarps = 8;
+      }
+      m = __reduce_max_sync(0xFFFFFFFFu, m);
+      if ((t & 31) == 0) s_red[t >> 5] = m;
+      if (nwarps == 8) {
+        asm volatile("bar.sync 3, %0;" ::"n"(XMAX_THREADS) : "memory");
+      } else {
+        xq_sync();
+      }
+      if (t == 0) {
+        uint32_t mm = 0;
+        for (int w = 0; w < nwarps; ++w) mm = max(mm, s_red[w]);
+        const float amax = __uint_as_float(mm);
+        float g = (amax == 0.0f) ? 1.0f : __fdiv_rn(2688.0f, amax);
+        if (!isfinite(g)) g = 1.0f;
+        *s_gx = g;
+      }
+    }
+    xq_sync();
+    const float g = *s_gx;
+    {
+      const float ds = ptx::e4m3_value(static_cast<uint32_t>(t));
+      s_rtab[t] = (ds == 0.0f) ? 0.0f : __fdiv_rn(g, ds);  // r = 0 keeps only signs
+    }
+    if (t == 0 && blockIdx.x == 0 && p.x_global_out != nullptr) *p.x_global_out = g;
+    xq_sync();
+    if (t == 0) ptx::mbar_arrive(g_ready);
+    uint32_t stage = 0, phase = 0;
+    const int nblk = p.M * 16;  // (token, 16-element block) pairs of one k-tile
+    WorkIter it;
+    for (it.start(p); it.sg.valid; it.next(p)) {
+      // every thread waits; all of them go on only if all saw the data
+      const bool landed = wait_bounded(&full[stage], phase, abort_flag, kFaultProducer, lim);
+      uint8_t* st = smem + stage * C::STAGE_BYTES;
+      const uint16_t* xr = reinterpret_cast<const uint16_t*>(st + C::XRAW_OFF);  // [XR][256]
+      const uint32_t codes = ptx::smem_u32(st + C::A_BYTES);
+      uint8_t* sfx = st + C::A_BYTES + C::B_BYTES + C::SFA_BYTES;
+      const int kcol0 = it.kt * BK;
+      for (int i = t; landed && i < nblk; i += XQ_THREADS) {
+        const int r = i >> 4, b = i & 15;
+        uint32_t c0 = 0u, c1 = 0u, sc = 0u;
+        if (kcol0 + 16 * b < p.K) {  // K % 16 == 0: a block is in range or past K
+          const uint4 v0 = *reinterpret_cast<const uint4*>(xr + r * BK + 16 * b);
+          const uint4 v1 = *reinterpret_cast<const uint4*>(xr + r * BK + 16 * b + 8);
+          const uint32_t mb = max(quant::absmax_bits8(v0), quant::absmax_bits8(v1));
+          sc = ptx::cvt_e4m3(__fmul_rn(quant::div6_rn(__uint_as_float(mb << 16)), g));
+          const float rs = s_rtab[sc];
+          float f[8];
+          f[0] = __fmul_rn(quant::bf16_lo(v0.x), rs);
+          f[1] = __fmul_rn(quant::bf16_hi(v0.x), rs);
+          f[2] = __fmul_rn(quant::bf16_lo(v0.y), rs);
+          f[3] = __fmul_rn(quant::bf16_hi(v0.y), rs);
+          f[4] = __fmul_rn(quant::bf16_lo(v0.z), rs);
+          f[5] = __fmul_rn(quant::bf16_hi(v0.z), rs);
+          f[6] = __fmul_rn(quant::bf16_lo(v0.w), rs);
+          f[7] = __fmul_rn(quant::bf16_hi(v0.w), rs);
+          c0 = ptx::cvt_e2m1x8(f);
+          f[0] = __fmul_rn(quant::bf16_lo(v1.x), rs);
+          f[1] = __fmul_rn(quant::bf16_hi(v1.x), rs);
+          f[2] = __fmul_rn(quant::bf16_lo(v1.y), rs);
+          f[3] = __fmul_rn(quant::bf16_hi(v1.y), rs);
+          f[4] = __fmul_rn(quant::bf16_lo(v1.z), rs);
+          f[5] = __fmul_rn(quant::bf16_hi(v1.z), rs);
+          f[6] = __fmul_rn(quant::bf16_lo(v1.w), rs);
+          f[7] = __fmul_rn(quant::bf16_hi(v1.w), rs);
+          c1 = ptx::cvt_e2m1x8(f);
+        }
+        // codes: bytes [8b, 8b+8) of token row r (128 bytes), 16-byte chunk
+        // b/2 at chunk (b/2) ^ (r % 8): the TMA's 128-byte swizzle
+        const uint32_t chunk = static_cast<uint32_t>(b >> 1) ^ static_cast<uint32_t>(r & 7);
+        ptx::st_shared_v2(codes + static_cast<uint32_t>(r) * 128u + (chunk << 4) +
+                              8u * static_cast<uint32_t>(b & 1),
+                          c0, c1);
+        // scale: atom b/4 (K = 64 step), line r % 32, byte group r / 32, block b % 4
+        sfx[(b >> 2) * 512 + (r & 31) * 16 + (r >> 5) * 4 + (b & 3)] = static_cast<uint8_t>(sc);
+      }
+      ptx::fence_proxy_async_smem();  // the MMA and tcgen05.cp read the stage through the async proxy
+      if (!xq_sync_and(landed)) break;
+      if (t == 0) ptx::mbar_arrive(&xready[stage]);
+      if (++stage == C::STAGES) {
+        stage = 0;
+        phase ^= 1u;
       }
     }
   }

@@ -661,7 +661,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const Unit unit = unit_of(t, p);
       int mb, nb;
       tile_coords(unit.tile, p, mb, nb);
-      if (!wait_bounded(tmem_full, acc_phase, ab, kFaultEpilogue)) break;
+      // warp-uniform: no lane may leave while the others go on to the
+      // warp-wide tensor-memory loads
+      if (!__all_sync(0xFFFFFFFFu, wait_bounded(tmem_full, acc_phase, ab, kFaultEpilogue))) break;
       ptx::tc_fence_after();
       if (p.fused == kFusedBf16Amax) {
         // gate columns [64 half, +64) and the matching up columns (+128) ->

@@ -531,27 +531,38 @@ nvfp4_status encode_sf(PFN_cuTensorMapEncodeTiled_v12000 enc, CUtensorMap* map, 
   return r == CUDA_SUCCESS ? NVFP4_OK : NVFP4_ERR_CUDA;
 }
 
-template <int BNT>
+template <int BNT, bool FUSED>
 nvfp4_status launch_skinny(DeviceState* st, int bit, const CUtensorMap& tmW, const CUtensorMap& tmX,
                            const CUtensorMap& tmSFW, const CUtensorMap& tmSFX,
                            const nvfp4::skinny::Params& p, int grid, cudaStream_t s) {
-  using nvfp4::skinny::Cfg;
+  using C = nvfp4::skinny::Cfg<BNT, FUSED>;
   {
     std::lock_guard<std::mutex> lock(g_mutex);
     if (!(st->skinny_smem_set & (1u << bit))) {
-      if (cudaFuncSetAttribute(nvfp4::skinny::skinny_kernel<BNT>,
+      if (cudaFuncSetAttribute(nvfp4::skinny::skinny_kernel<BNT, FUSED>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(Cfg<BNT>::SMEM_BYTES)) != cudaSuccess) {
+                               static_cast<int>(C::SMEM_BYTES)) != cudaSuccess) {
         cudaGetLastError();
         return NVFP4_ERR_CUDA;
       }
       st->skinny_smem_set |= 1u << bit;
     }
   }
-  return launch_pdl(nvfp4::skinny::skinny_kernel<BNT>, static_cast<unsigned>(grid),
-                    nvfp4::skinny::NUM_THREADS, Cfg<BNT>::SMEM_BYTES, s, 1u, tmW, tmX, tmSFW,
-                    tmSFX, p);
+  return launch_pdl(nvfp4::skinny::skinny_kernel<BNT, FUSED>, static_cast<unsigned>(grid),
+                    C::THREADS, C::SMEM_BYTES, s, 1u, tmW, tmX, tmSFW, tmSFX, p);
 }
+
+// Tokens quantized inside the few-token GEMM (nvfp4_linear, m <= XR = 8): the
+// bf16 X, and where its global comes from (static, amax partials, or the
+// kernel's own max over X of at most kSelfAmaxBytes).
+struct XFused {
+  const void* x;
+  int64_t ldx;
+  const float* global_in;
+  const float* partials;
+  int nparts;
+  float* global_out;
+};
 
 // Few tokens (m <= 64): Y^T = B A^T with the weights on the MMA's 128-row
 // side and the tokens as its N; stream-K across all SMs when the weight tiles
@@ -565,19 +576,43 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
                          const uint8_t* b_codes, const uint8_t* b_sf, const float* b_global,
                          void* y, int y_dtype, int64_t ldy, int64_t m, int64_t n, int64_t k,
                          void* workspace, size_t workspace_bytes, bool zero_counters,
-                         int early_w, cudaStream_t s, int stall = 0, uint64_t limit_ns = 0) {
+                         int early_w, cudaStream_t s, int stall = 0, uint64_t limit_ns = 0,
+                         const XFused* xf = nullptr) {
   using namespace nvfp4::skinny;
   const int bnt = m <= 16 ? 16 : m <= 32 ? 32 : 64;  // callers route m <= 64 here
+  if (xf != nullptr && m > XR) return NVFP4_ERR_UNSUPPORTED;
   CUtensorMap tmW, tmX, tmSFW, tmSFX;
   if (nvfp4_status e = encode_2d(enc, &tmW, b_codes, static_cast<uint64_t>(k / 2),
                                  static_cast<uint64_t>(n), BW))
     return e;
-  if (nvfp4_status e = encode_2d(enc, &tmX, a_codes, static_cast<uint64_t>(k / 2),
-                                 static_cast<uint64_t>(m), static_cast<uint32_t>(bnt)))
-    return e;
   if (nvfp4_status e = encode_sf(enc, &tmSFW, b_sf, n, k, 1u)) return e;
-  if (nvfp4_status e = encode_sf(enc, &tmSFX, a_sf, m, k, 1u)) return e;
+  if (xf != nullptr) {
+    // bf16 token tiles of [XR][256] (rows past m and columns past k zero-filled)
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(k), static_cast<cuuint64_t>(m)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(xf->ldx) * 2u};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(BK), static_cast<cuuint32_t>(XR)};
+    cuuint32_t estr[2] = {1u, 1u};
+    if (enc(&tmX, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(xf->x), dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return NVFP4_ERR_CUDA;
+    tmSFX = tmSFW;  // not read in this mode
+  } else {
+    if (nvfp4_status e = encode_2d(enc, &tmX, a_codes, static_cast<uint64_t>(k / 2),
+                                   static_cast<uint64_t>(m), static_cast<uint32_t>(bnt)))
+      return e;
+    if (nvfp4_status e = encode_sf(enc, &tmSFX, a_sf, m, k, 1u)) return e;
+  }
   Params p;
+  std::memset(&p, 0, sizeof p);
+  if (xf != nullptr) {
+    p.x = static_cast<const uint16_t*>(xf->x);
+    p.ldx = xf->ldx;
+    p.x_global_in = xf->global_in;
+    p.x_partials = xf->partials;
+    p.x_nparts = xf->nparts;
+    p.x_global_out = xf->global_out;
+  }
   p.M = static_cast<int>(m);
   p.N = static_cast<int>(n);
   p.K = static_cast<int>(k);
@@ -613,10 +648,13 @@ nvfp4_status gemm_skinny(PFN_cuTensorMapEncodeTiled_v12000 enc, DeviceState* st,
     }
   }
   nvfp4_status e;
+  if (xf != nullptr) {
+    return launch_skinny<16, true>(st, 3, tmW, tmX, tmSFW, tmSFX, p, grid, s);
+  }
   switch (bnt) {
-    case 16: e = launch_skinny<16>(st, 0, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
-    case 32: e = launch_skinny<32>(st, 1, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
-    default: e = launch_skinny<64>(st, 2, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    case 16: e = launch_skinny<16, false>(st, 0, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    case 32: e = launch_skinny<32, false>(st, 1, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
+    default: e = launch_skinny<64, false>(st, 2, tmW, tmX, tmSFW, tmSFX, p, grid, s); break;
   }
   return e;
 }
@@ -820,6 +858,30 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   uint8_t* a_sf = a_codes + round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);
   float* a_global = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(m, k), 256));
   float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a_global) + 256);
+  if (m <= nvfp4::skinny::XR) {
+    // A decode step's few tokens are quantized inside the GEMM (bit for bit
+    // as nvfp4_quantize): no quantizer kernel sits between the previous
+    // layer and this GEMM. A dynamic global over X above kSelfAmaxBytes
+    // still takes the amax pass first (its partials are order-free). Every
+    // CTA quantizes its k-range of all m tokens, so the redundant work grows
+    // with m: measured on graphs of decode steps, 1 and 8 tokens gained
+    // 0.6-1.0 us per step, 16 tokens and more lost 1.4-9 us.
+    using namespace nvfp4::quant;
+    XFused xf{x, ldx, x_global, nullptr, 0, a_global};
+    if (x_global == nullptr && m * k * 2 > kSelfAmaxBytes) {
+      if (nvfp4_status e = quant_occupancy(st)) return e;
+      const int threads = amax_threads(m, k);
+      const int64_t blocks = amax_blocks(m, k, ldx, st, threads);
+      if (blocks > kMaxPartials) return NVFP4_ERR_UNSUPPORTED;
+      amax_kernel<<<static_cast<unsigned>(blocks), threads, 0, s>>>(
+          static_cast<const uint16_t*>(x), m, k, ldx, partials);
+      if (nvfp4_status e = launch_status()) return e;
+      xf.partials = partials;
+      xf.nparts = static_cast<int>(blocks);
+    }
+    return gemm_skinny(enc, st, a_codes, a_sf, a_global, w_codes, w_sf, w_global, y, y_dtype, ldy,
+                       m, n, k, w, skinny_workspace_bytes(m, n), false, 1, s, 0, 0, &xf);
+  }
   // the quantized X is private to this call: its padding rows' scales are
   // not written (only the GEMM reads them, against zero-filled codes)
   if (nvfp4_status e = quantize_launch(x, m, k, ldx, x_global, a_codes, a_sf, a_global, partials,

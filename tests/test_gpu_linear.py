@@ -35,7 +35,7 @@ def counter_bytes(n):
     return -(-(4 * max(4 * -(-n // 128), 64 * 16)) // 256) * 256
 
 
-@pytest.mark.parametrize("m", [1, 8, 16, 33, 64, 65, 300])
+@pytest.mark.parametrize("m", [1, 8, 16, 17, 32, 33, 64, 65, 300])
 @pytest.mark.parametrize("static", [False, True])
 def test_linear_equals_quantize_then_gemm(nv, orc, m, static):
     """Few-token (m <= 64, K split) and paired (m > 64) GEMMs behind the
@@ -64,6 +64,35 @@ def test_linear_equals_quantize_then_gemm(nv, orc, m, static):
         gemm_check(y, ref, norms(orc, qx), norms(orc, qw), f"linear m={m} static={static} {dt}")
     if m <= 64:
         assert int(ws[:counter_bytes(n)].count_nonzero()) == 0, "split counters not reset"
+    assert nv.read_fault() == 0
+
+
+@pytest.mark.parametrize("m,k", [(8, 4096), (7, 2336), (8, 5120), (2, 65536)])
+@pytest.mark.parametrize("static", [False, True])
+def test_linear_in_kernel_token_quantization(nv, orc, m, k, static):
+    """At most 8 tokens are quantized inside the few-token GEMM. Its dynamic
+    global comes from the kernel's own max over X up to 64 KiB of bf16 (8 x
+    4096: exactly the bound; 7 x 2336: a ragged last k-tile), from the amax
+    pass's partials above that (8 x 5120, 2 x 65536), or from a static
+    global; every way equals quantize + GEMM bit for bit, and the oracle
+    within the tolerance."""
+    n = 640
+    x = gaussian(m, k, 31 * m + k)
+    qw = orc.quantize(bits(gaussian(n, k, 32, 0.02)))
+    W = upload(qw)
+    g = None
+    if static:
+        g = torch.tensor([float(orc.global_from_amax(orc.tensor_amax(bits(x)) * 1.25))],
+                         dtype=torch.float32, device="cuda")
+    xd = x.cuda()
+    y = nv.linear(xd, W, out_dtype=torch.float32, global_scale=g,
+                  workspace=nv.linear_workspace(m, n, k))
+    gws = torch.empty(nv.gemm_workspace_bytes(m, n, k), dtype=torch.uint8, device="cuda")
+    y2 = nv.gemm(nv.quantize(xd, global_scale=g), W, out_dtype=torch.float32, workspace=gws)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2), (m, k, static)
+    qx = orc.quantize(bits(x), None if g is None else np.float32(g.item()))
+    gemm_check(y, orc.gemm(qx, qw), norms(orc, qx), norms(orc, qw), f"in-kernel m={m} k={k}")
     assert nv.read_fault() == 0
 
 
