@@ -16,15 +16,16 @@
 //   warp 0  TMA producer (both CTAs): A (128 rows x 128 B) and B (128 N rows x
 //           128 B) with 128-byte swizzle, this CTA's A scale atoms and all 256
 //           B-row scale atoms, into a 5-stage ring. Both CTAs' copies signal
-//           the even CTA's full barrier, which expects the pair's bytes.
+//           the even CTA's barriers, which expect the pair's bytes: the scale
+//           atoms (requested first) one barrier, the A and B tiles another.
 //   warp 1  allocates 512 tensor-memory columns in both CTAs; in the even CTA
 //           one thread issues 4 MMAs (kind::mxf4nvf4.block16, K = 64) per
 //           256-element k-tile, then commits to the empty barrier of both
 //           CTAs and to the scale buffer's empty barrier.
 //   warps 2, 3  (even CTA) copy each stage's scale atoms into that stage's
 //           tensor-memory scale buffer (one per ring stage; tcgen05.cp
-//           32x128b.warpx4, both CTAs), 6 of the 12 copies each, and commit
-//           to the buffer's full barrier. Each tcgen05.cp costs a fixed ~50
+//           32x128b.warpx4, both CTAs) as soon as the atoms land, 6 of the 12
+//           copies each, and commit to the buffer's full barrier. Each tcgen05.cp costs a fixed ~50
 //           cycles whatever its size; issued from the MMA thread the 12 copies
 //           per k-tile serialise with the 4 MMAs (measured 4302 -> 2803 TF/s),
 //           and one copy warp alone issues slower than the MMAs consume.
@@ -399,7 +400,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   uint64_t* drain = tmem_empty + 1;
   uint64_t* sf_full = drain + 1;
   uint64_t* drain_sf = sf_full + NSF;
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain_sf + 1);
+  // a stage's scale atoms land on their own barrier, ahead of its A and B
+  // tiles: the copy warps move them into tensor memory while the operand
+  // tiles are still in flight
+  uint64_t* sf_landed = drain_sf + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sf_landed + STAGES);
   volatile uint32_t* abort_flag = tmem_holder + 1;
   uint32_t* h_max = tmem_holder + 2;  // kFusedBf16Amax: max|h| bits over the CTA
 
@@ -414,6 +419,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       ptx::mbar_init(&full[s], 1);
       ptx::mbar_init(&empty[s], 1);
+      ptx::mbar_init(&sf_landed[s], 1);
     }
     ptx::mbar_init(tmem_full, 1);
     ptx::mbar_init(tmem_empty, 2 * NUM_EPI_WARPS);
@@ -472,22 +478,30 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (++it.kt == it.k1) it = first(it.t + num_pairs);
         return it;
       };
-      // the even CTA's barrier counts both CTAs' bytes of a stage
+      // the even CTA's barriers count both CTAs' bytes of a stage: scale
+      // atoms on sf_landed (requested first), A and B tiles on full
       auto load_b = [&](const Item& it, uint32_t s) {
         uint8_t* st = smem + s * STAGE_BYTES;
-        const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
-        ptx::tma_load_2d_pair(st + A_BYTES, &tmB, bar, it.kt * BK_BYTES,
-                              it.nb * BN + static_cast<int>(rank) * HALF);
-        ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tmSFB, bar, 0, it.kt * 4,
+        ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES + SFA_BYTES, &tmSFB,
+                              ptx::mapa_shared(ptx::smem_u32(&sf_landed[s]), 0), 0, it.kt * 4,
                               it.nb * 2);
+        ptx::tma_load_2d_pair(st + A_BYTES, &tmB, ptx::mapa_shared(ptx::smem_u32(&full[s]), 0),
+                              it.kt * BK_BYTES, it.nb * BN + static_cast<int>(rank) * HALF);
       };
       auto load_a = [&](const Item& it, uint32_t s) {
         uint8_t* st = smem + s * STAGE_BYTES;
-        const uint32_t bar = ptx::mapa_shared(ptx::smem_u32(&full[s]), 0);
-        ptx::tma_load_2d_pair(st, &tmA, bar, it.kt * BK_BYTES,
-                              it.mb * BM + static_cast<int>(rank) * HALF);
-        ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES, &tmSFA, bar, 0, it.kt * 4,
+        ptx::tma_load_3d_pair(st + A_BYTES + B_BYTES, &tmSFA,
+                              ptx::mapa_shared(ptx::smem_u32(&sf_landed[s]), 0), 0, it.kt * 4,
                               it.mb * 2 + static_cast<int>(rank));
+        ptx::tma_load_2d_pair(st, &tmA, ptx::mapa_shared(ptx::smem_u32(&full[s]), 0),
+                              it.kt * BK_BYTES, it.mb * BM + static_cast<int>(rank) * HALF);
+      };
+      // both barriers of a stage are armed by the even CTA for the pair
+      auto arm = [&](uint32_t s) {
+        if (leader) {
+          ptx::mbar_arrive_expect_tx(&sf_landed[s], 2 * (SFA_BYTES + SFB_BYTES));
+          ptx::mbar_arrive_expect_tx(&full[s], 2 * (A_BYTES + B_BYTES));
+        }
       };
       Item it = first(pair);
       // The ring's first pass needs no empty-slot wait; with early_w its B
@@ -495,7 +509,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       int npre = 0;
       if (p.early_w) {
         for (Item w = it; npre < STAGES && w.t < num_units; ++npre, w = next(w)) {
-          if (leader) ptx::mbar_arrive_expect_tx(&full[npre], 2 * STAGE_BYTES);
+          arm(static_cast<uint32_t>(npre));
           load_b(w, static_cast<uint32_t>(npre));
         }
       }
@@ -520,7 +534,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           continue;
         }
-        if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+        arm(stage);
         load_a(it, stage);
         load_b(it, stage);
         pending |= 1u << stage;
@@ -536,7 +550,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // else waits for them. Without one the MMA thread consumes the same
         // phases, so these waits end as soon as the last copies land.
         for (int s = 0; s < STAGES; ++s)
-          if (pending & (1u << s)) drain_wait(&full[s], (pending_parity >> s) & 1u);
+          if (pending & (1u << s)) {
+            drain_wait(&sf_landed[s], (pending_parity >> s) & 1u);
+            drain_wait(&full[s], (pending_parity >> s) & 1u);
+          }
       }
     }
   } else if (warp == 1) {
@@ -598,10 +615,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int t = pair; t < num_units && !aborted; t += num_pairs) {
         const Unit w = unit_of(t, p);
         for (int kt = w.k0; kt < w.k1; ++kt) {
-          // The stage's data having landed also means the MMAs of its previous
-          // use finished (the producer waited for them before reloading it),
-          // so scale buffer `stage` is free: no wait on the MMA thread here.
-          if (!wait_bounded(&full[stage], phase, ab, kFaultScales)) {
+          // The stage's scale atoms having landed also means the MMAs of its
+          // previous use finished (the producer waited for them before
+          // reloading it), so scale buffer `stage` is free: no wait on the
+          // MMA thread here.
+          if (!wait_bounded(&sf_landed[stage], phase, ab, kFaultScales)) {
             aborted = true;
             break;
           }
