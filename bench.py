@@ -302,8 +302,11 @@ def make_inputs(name: str, rank: int = 0) -> dict:
         cfg = wl.decode(m, k, n)
         cfg.x_seed = rank_x_seed(rank)
         return dict(kind="decode", x=cfg.x(), w=cfg.w(), m=m, n=n, k=k, gemms=[(m, n, k)],
-                    desc=(f"decode: X {m}x{k} bf16 ~N(0,1) -> nvfp4_linear (quantize, then the "
-                          f"W4A4 GEMM launched to overlap it) vs W {n}x{k} ~N(0,0.02) NVFP4"))
+                    desc=(f"decode: X {m}x{k} bf16 ~N(0,1) -> nvfp4_linear ("
+                          + ("tokens quantized inside the few-token W4A4 GEMM"
+                             if m <= 8 else
+                             "quantize, then the W4A4 GEMM launched to overlap it")
+                          + f") vs W {n}x{k} ~N(0,0.02) NVFP4"))
     raise SystemExit(f"unknown workload {name}")
 
 
@@ -700,7 +703,12 @@ class DecodeRun:
         self.Aq = nv.NVFP4Tensor.empty(m, k)
         self.A, self.y = self.As[0], self.ys[0]   # what the oracle leg samples
         one_pass = m * k * 2 <= nv.ONE_PASS_MAX_BYTES
-        self.launches_per_step = 2 if one_pass else 3
+        if m <= nv.LINEAR_IN_KERNEL_MAX_TOKENS:
+            # the tokens are quantized inside the few-token GEMM; a dynamic
+            # global over X above the one-pass bound adds the amax pass
+            self.launches_per_step = 1 if one_pass else 2
+        else:
+            self.launches_per_step = 2 if one_pass else 3
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):      # eager run of every call before capture
             self._linear_all()
@@ -777,11 +785,15 @@ def measure_decode(wk, stream, steps, warmup, pk, dist=None):
     gemm_bytes = n * k // 2 + n * k // 16 + m * k // 2 + m * k // 16 + m * n * 2
     roof = {"bound": "hbm", "achieved": round(gbs, 1), "peak": pk["hbm_gbs"], "unit": "GB/s",
             "frac": round(gbs / pk["hbm_gbs"], 4), "traffic": dram_traffic(wk["name"]),
-            "kernel": ("nvfp4_linear step: quantize_kernel (" +
-                       ("takes the max itself" if run.launches_per_step == 2 else
-                        "after amax_kernel") + ") + " +
-                       ("skinny_kernel" if m <= 64 else "gemm_kernel") +
-                       ", back to back over rotating weight copies"),
+            "kernel": (("nvfp4_linear step: " + ("" if run.launches_per_step == 1 else
+                                                  "amax_kernel + ") +
+                        "skinny_kernel with in-kernel token quantization")
+                       if m <= nvfp4.LINEAR_IN_KERNEL_MAX_TOKENS else
+                       ("nvfp4_linear step: quantize_kernel (" +
+                        ("takes the max itself" if run.launches_per_step == 2 else
+                         "after amax_kernel") + ") + " +
+                        ("skinny_kernel" if m <= 64 else "gemm_kernel")))
+                      + ", back to back over rotating weight copies",
             "peak_source": f"measured copy bandwidth ({pk['source']})",
             "algorithmic_bytes_per_launch": step_bytes,
             "gemm_alone_us": round(gemm_ms * 1e3, 2),

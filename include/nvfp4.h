@@ -233,7 +233,8 @@ size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * nvfp4_quantize of X into the workspace followed by nvfp4_gemm, with
  * identical results. The GEMM is launched to start while the quantizer runs:
  * its set-up and its first weight tiles overlap the quantization. For at
- * most 8 tokens there is no quantizer kernel: the few-token GEMM quantizes
+ * most NVFP4_LINEAR_IN_KERNEL_MAX_TOKENS (8) tokens there is no quantizer
+ * kernel: the few-token GEMM quantizes
  * each k-tile of X as it lands in shared memory (same arithmetic, same
  * bits), after an amax pass only when the global is dynamic and X exceeds
  * NVFP4_ONE_PASS_MAX_BYTES. This relies on W, w_sf and w_global being
@@ -260,6 +261,7 @@ size_t nvfp4_linear_workspace_bytes(int64_t m, int64_t n, int64_t k);
  * Errors: INVALID_ARG (null pointer, bad size, short workspace), MISALIGNED,
  * UNSUPPORTED (k % 32 != 0, sizes >= 2^31), CUDA.
  */
+#define NVFP4_LINEAR_IN_KERNEL_MAX_TOKENS 8
 nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
                           const float* x_global, const uint8_t* w_codes,
                           const uint8_t* w_sf, const float* w_global, int64_t n,

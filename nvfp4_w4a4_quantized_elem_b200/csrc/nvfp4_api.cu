@@ -858,6 +858,7 @@ nvfp4_status nvfp4_linear(const void* x, int64_t m, int64_t k, int64_t ldx,
   uint8_t* a_sf = a_codes + round_up(static_cast<size_t>(m) * static_cast<size_t>(k / 2), 256);
   float* a_global = reinterpret_cast<float*>(a_sf + round_up(nvfp4_sf_bytes(m, k), 256));
   float* partials = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(a_global) + 256);
+  static_assert(nvfp4::skinny::XR == NVFP4_LINEAR_IN_KERNEL_MAX_TOKENS, "header and kernel agree");
   if (m <= nvfp4::skinny::XR) {
     // A decode step's few tokens are quantized inside the GEMM (bit for bit
     // as nvfp4_quantize): no quantizer kernel sits between the previous

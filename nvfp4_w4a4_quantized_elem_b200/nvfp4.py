@@ -20,6 +20,9 @@ LIB_PATH = os.path.join(_HERE, "libnvfp4.so")
 # Dynamic quantization of x with rows * k * 2 bytes up to this bound runs
 # one kernel (NVFP4_ONE_PASS_MAX_BYTES of nvfp4.h): no amax pass.
 ONE_PASS_MAX_BYTES = 65536
+# nvfp4_linear quantizes at most this many tokens inside the few-token GEMM
+# (NVFP4_LINEAR_IN_KERNEL_MAX_TOKENS of nvfp4.h)
+LINEAR_IN_KERNEL_MAX_TOKENS = 8
 
 NVFP4_OK = 0
 STATUS_NAMES = {0: "NVFP4_OK", 1: "NVFP4_ERR_INVALID_ARG", 2: "NVFP4_ERR_UNSUPPORTED",

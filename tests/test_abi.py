@@ -38,6 +38,8 @@ def test_binding_constants_match_the_header():
     text = open(HEADER).read()
     m = re.search(r"#define NVFP4_ONE_PASS_MAX_BYTES (\d+)", text)
     assert m and int(m.group(1)) == nvfp4.ONE_PASS_MAX_BYTES
+    m = re.search(r"#define NVFP4_LINEAR_IN_KERNEL_MAX_TOKENS (\d+)", text)
+    assert m and int(m.group(1)) == nvfp4.LINEAR_IN_KERNEL_MAX_TOKENS
 
 
 def test_library_exports_every_declared_symbol(L):
