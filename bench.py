@@ -788,7 +788,7 @@ def measure_decode(wk, stream, steps, warmup, pk, dist=None):
             "kernel": (("nvfp4_linear step: " + ("" if run.launches_per_step == 1 else
                                                   "amax_kernel + ") +
                         "skinny_kernel with in-kernel token quantization")
-                       if m <= nvfp4.LINEAR_IN_KERNEL_MAX_TOKENS else
+                       if m <= nv.LINEAR_IN_KERNEL_MAX_TOKENS else
                        ("nvfp4_linear step: quantize_kernel (" +
                         ("takes the max itself" if run.launches_per_step == 2 else
                          "after amax_kernel") + ") + " +
