@@ -74,7 +74,10 @@ constexpr uint64_t kDrainLimitNs = 100000000ull;
 constexpr size_t kSmemPerCta = 220 * 1024;
 constexpr int kMaxSplits = 8;     // stream-K: at most this many CTAs per weight tile
 constexpr int kMaxContrib = kMaxSplits + 1;  // contributor slots per tile (host-checked)
-constexpr int kSumTokens = 8;     // tokens summed per round of slab loads
+// tokens summed per round of slab loads: every load of a round is issued
+// before its first add, so a round costs one L2 round trip
+template <int BNT, bool FUSED>
+__host__ __device__ constexpr int sum_tokens() { return FUSED || BNT == 16 ? 8 : 16; }
 
 enum : uint32_t { kFaultProducer = 16u, kFaultMma = 32u, kFaultEpilogue = 64u, kFaultScales = 128u };
 
@@ -271,22 +274,22 @@ struct WorkIter {
   }
 };
 
-// One output column of a stream-K tile for kSumTokens tokens from m0: the
+// One output column of a stream-K tile for T tokens from m0: the
 // NC contributors' FP32 slabs ([M][BW] each, `slab` floats apart) added in
 // contributor (= k) order. Every load is issued before the first add, so a
 // round costs one L2 round trip rather than one per contributor; rows past M
 // are clamped to a valid row and their sums are not stored.
-template <int NC>
+template <int NC, int T>
 __device__ __forceinline__ void sum_slabs(const float* col, int64_t slab, int m0, int M,
-                                          float (&acc)[kSumTokens]) {
-  float v[NC][kSumTokens];
+                                          float (&acc)[T]) {
+  float v[NC][T];
 #pragma unroll
   for (int j = 0; j < NC; ++j)
 #pragma unroll
-    for (int i = 0; i < kSumTokens; ++i)
+    for (int i = 0; i < T; ++i)
       v[j][i] = __ldcg(col + j * slab + static_cast<int64_t>(min(m0 + i, M - 1)) * BW);
 #pragma unroll
-  for (int i = 0; i < kSumTokens; ++i) {
+  for (int i = 0; i < T; ++i) {
     float a = v[0][i];
 #pragma unroll
     for (int j = 1; j < NC; ++j) a += v[j][i];
@@ -632,21 +635,22 @@ __global__ void __launch_bounds__(Cfg<BNT, FUSED>::THREADS, 1)
           if (n_ok) {
             const float* col = p.partial + static_cast<int64_t>(wt) * kMaxContrib * p.M * BW + nl;
             const int64_t slab_len = static_cast<int64_t>(p.M) * BW;
-            for (int m0 = 0; m0 < p.M; m0 += kSumTokens) {
-              float acc[kSumTokens];
+            constexpr int T = sum_tokens<BNT, FUSED>();
+            for (int m0 = 0; m0 < p.M; m0 += T) {
+              float acc[T];
               switch (n_contrib) {
-                case 1: sum_slabs<1>(col, slab_len, m0, p.M, acc); break;
-                case 2: sum_slabs<2>(col, slab_len, m0, p.M, acc); break;
-                case 3: sum_slabs<3>(col, slab_len, m0, p.M, acc); break;
-                case 4: sum_slabs<4>(col, slab_len, m0, p.M, acc); break;
-                case 5: sum_slabs<5>(col, slab_len, m0, p.M, acc); break;
-                case 6: sum_slabs<6>(col, slab_len, m0, p.M, acc); break;
-                case 7: sum_slabs<7>(col, slab_len, m0, p.M, acc); break;
-                case 8: sum_slabs<8>(col, slab_len, m0, p.M, acc); break;
-                default: sum_slabs<kMaxContrib>(col, slab_len, m0, p.M, acc); break;
+                case 1: sum_slabs<1, T>(col, slab_len, m0, p.M, acc); break;
+                case 2: sum_slabs<2, T>(col, slab_len, m0, p.M, acc); break;
+                case 3: sum_slabs<3, T>(col, slab_len, m0, p.M, acc); break;
+                case 4: sum_slabs<4, T>(col, slab_len, m0, p.M, acc); break;
+                case 5: sum_slabs<5, T>(col, slab_len, m0, p.M, acc); break;
+                case 6: sum_slabs<6, T>(col, slab_len, m0, p.M, acc); break;
+                case 7: sum_slabs<7, T>(col, slab_len, m0, p.M, acc); break;
+                case 8: sum_slabs<8, T>(col, slab_len, m0, p.M, acc); break;
+                default: sum_slabs<kMaxContrib, T>(col, slab_len, m0, p.M, acc); break;
               }
 #pragma unroll
-              for (int i = 0; i < kSumTokens; ++i) {
+              for (int i = 0; i < T; ++i) {
                 if (m0 + i >= p.M) break;
                 const int64_t o = static_cast<int64_t>(m0 + i) * p.ldy + n;
                 if (p.y_fp32)
