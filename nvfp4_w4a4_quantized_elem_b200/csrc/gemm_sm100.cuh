@@ -753,6 +753,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int row0 = mb * BM + static_cast<int>(rank) * HALF + q * 32;  // this warp's rows
       const int col0 = nb * BN + half * 128;
       if (p.split > 1) {
+        // rows past M (a tile's padding): no partial, no count, no output
+        if (row0 >= p.M) continue;
         // this slice's partial -> its slab; the region's last slice sums all
         // slabs in slice order (whichever slice that is) and writes Y
         const int region = static_cast<int>(rank) * 8 + (warp - EPI_WARP0);
@@ -783,23 +785,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         last = __shfl_sync(0xFFFFFFFFu, last, 0);
         if (!last) continue;
         __threadfence();
-        if (row0 < p.M) {
-          // 32 columns at a time: all slices' loads first, then the adds
-          for (int cc = 0; cc < 4; ++cc) {
-            uint32_t acc[32];
-            const float4* src = reinterpret_cast<const float4*>(base) + lane + 32 * (8 * cc);
-            switch (p.split) {
-              case 2: sum_slices<2>(src, slab_stride / 4, acc); break;
-              case 3: sum_slices<3>(src, slab_stride / 4, acc); break;
-              default: sum_slices<kMaxSplitK>(src, slab_stride / 4, acc); break;
-            }
-            if (!p.y_fp32) {
-              emit([&](uint32_t b) { stage_bf16(b, lane, acc, alpha); }, col0 + 32 * cc, row0);
-            } else {
-              emit([&](uint32_t b) { stage_f32(b, lane, acc, 0, alpha); }, col0 + 32 * cc, row0);
-              emit([&](uint32_t b) { stage_f32(b, lane, acc, 16, alpha); }, col0 + 32 * cc + 16,
-                   row0);
-            }
+        // 32 columns at a time: all slices' loads first, then the adds
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t acc[32];
+          const float4* src = reinterpret_cast<const float4*>(base) + lane + 32 * (8 * cc);
+          switch (p.split) {
+            case 2: sum_slices<2>(src, slab_stride / 4, acc); break;
+            case 3: sum_slices<3>(src, slab_stride / 4, acc); break;
+            default: sum_slices<kMaxSplitK>(src, slab_stride / 4, acc); break;
+          }
+          if (!p.y_fp32) {
+            emit([&](uint32_t b) { stage_bf16(b, lane, acc, alpha); }, col0 + 32 * cc, row0);
+          } else {
+            emit([&](uint32_t b) { stage_f32(b, lane, acc, 0, alpha); }, col0 + 32 * cc, row0);
+            emit([&](uint32_t b) { stage_f32(b, lane, acc, 16, alpha); }, col0 + 32 * cc + 16,
+                 row0);
           }
         }
         if (lane == 0) *cnt = 0u;  // ready for the next call

@@ -96,6 +96,27 @@ def test_linear_in_kernel_token_quantization(nv, orc, m, k, static):
     assert nv.read_fault() == 0
 
 
+@pytest.mark.parametrize("m,k", [(1, 32), (3, 96), (8, 160), (5, 288), (12, 96)])
+def test_linear_short_k(nv, orc, m, k):
+    """K shorter than one 256-element k-tile, or one k-tile and a ragged
+    rest: the token tile's columns past K are zero-filled by the TMA and the
+    in-kernel quantizer writes zero codes and scales for their blocks (the
+    12-token case runs the separate quantizer for comparison)."""
+    n = 384
+    x = gaussian(m, k, 7 * m + k)
+    qw = orc.quantize(bits(gaussian(n, k, 8, 0.02)))
+    W = upload(qw)
+    xd = x.cuda()
+    y = nv.linear(xd, W, out_dtype=torch.float32, workspace=nv.linear_workspace(m, n, k))
+    gws = torch.empty(max(16, nv.gemm_workspace_bytes(m, n, k)), dtype=torch.uint8, device="cuda")
+    y2 = nv.gemm(nv.quantize(xd), W, out_dtype=torch.float32, workspace=gws)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2), (m, k)
+    qx = orc.quantize(bits(x))
+    gemm_check(y, orc.gemm(qx, qw), norms(orc, qx), norms(orc, qw), f"short k m={m} k={k}")
+    assert nv.read_fault() == 0
+
+
 def test_linear_strided_and_ragged_x(nv, orc):
     """x with a row pitch larger than k, and k not a multiple of 256 (the last
     k-tile of every slice is partial): linear equals the chain."""
