@@ -38,6 +38,12 @@
 //   warps 4-7  epilogue: each thread owns one weight row (= one output
 //              column n) and drains its BNT token values 32 at a time; for a
 //              fixed token the 32 lanes write 32 consecutive columns.
+//   warps 8-11 (in-kernel token quantization, m <= XR: nvfp4_linear of a
+//              decode step) the producer brings each k-tile of the bf16
+//              tokens instead of their codes and scales, and these warps
+//              quantize it into the stage (X's global first: static, from
+//              the amax pass's partials, or the max over X taken together
+//              with the epilogue warps); the MMA and copy warps wait for them.
 // Every wait is bounded; on expiry the fault word is set, copies and MMAs in
 // flight are drained (bounded) and tensor memory is freed before exit.
 #pragma once
