@@ -232,6 +232,16 @@ def job_throughput(flops_per_rank: float, world: int, ms_per_step: float) -> flo
     return flops_per_rank * world / (ms_per_step * 1e-3) / 1e12
 
 
+def linear_launches(m: int, k: int, static_global: bool) -> int:
+    """Kernels one nvfp4_linear call launches (the library's dispatch): at
+    most LINEAR_IN_KERNEL_MAX_TOKENS tokens are quantized inside the GEMM;
+    a dynamic global over X above ONE_PASS_MAX_BYTES adds the amax pass."""
+    from nvfp4_w4a4_quantized_elem_b200 import nvfp4 as nv
+    amax_pass = (not static_global) and m * k * 2 > nv.ONE_PASS_MAX_BYTES
+    quantizer = m > nv.LINEAR_IN_KERNEL_MAX_TOKENS
+    return 1 + int(quantizer) + int(amax_pass)
+
+
 def decode_rotation(weight_bytes: int) -> int:
     """Weight copies a decode run rotates over: their total is at least 3x
     L2, so a step's weights were evicted by the others' since its last use."""
@@ -377,7 +387,7 @@ class Step:
             if nb:
                 self.gws = torch.zeros(nb, dtype=torch.uint8, device=dev)
             self.lws = nvfp4.linear_workspace(m, n, k, dev)
-            self.launches = 2 if (wk.get("x_global") is not None or one_pass) else 3
+            self.launches = linear_launches(m, k, wk.get("x_global") is not None)
             self.nphases = 2
         else:
             ffn = wk["ffn"]
@@ -702,13 +712,7 @@ class DecodeRun:
         self.gstatic = torch.full((1,), 7.0, dtype=torch.float32, device="cuda")
         self.Aq = nv.NVFP4Tensor.empty(m, k)
         self.A, self.y = self.As[0], self.ys[0]   # what the oracle leg samples
-        one_pass = m * k * 2 <= nv.ONE_PASS_MAX_BYTES
-        if m <= nv.LINEAR_IN_KERNEL_MAX_TOKENS:
-            # the tokens are quantized inside the few-token GEMM; a dynamic
-            # global over X above the one-pass bound adds the amax pass
-            self.launches_per_step = 1 if one_pass else 2
-        else:
-            self.launches_per_step = 2 if one_pass else 3
+        self.launches_per_step = linear_launches(m, k, static_global=False)
         torch.cuda.synchronize()
         with torch.cuda.stream(stream):      # eager run of every call before capture
             self._linear_all()

@@ -112,3 +112,17 @@ def test_clock_sample_uses_nvidia_smi_timestamp():
     assert abs(t - (time.mktime(time.strptime("2026/12/02 21:25:18", "%Y/%m/%d %H:%M:%S")) + 0.25)) < 1e-6
     assert rest.startswith("0, 1700, 1965")
     assert bench.ClockSampler.parse("no stamp, 0, 1700", arrival=123.0) == (123.0, "0, 1700")
+
+
+def test_linear_launch_count_follows_the_dispatch():
+    """gpu_launches of the decode and linear lines: one kernel for at most 8
+    tokens (quantized inside the GEMM), plus the quantizer above 8 tokens,
+    plus the amax pass for a dynamic global over more than 64 KiB of X."""
+    assert bench.linear_launches(1, 5120, False) == 1
+    assert bench.linear_launches(8, 4096, False) == 1      # exactly 64 KiB
+    assert bench.linear_launches(8, 5120, False) == 2      # amax pass
+    assert bench.linear_launches(8, 5120, True) == 1       # static global
+    assert bench.linear_launches(9, 2048, False) == 2      # quantizer takes the max
+    assert bench.linear_launches(32, 5120, False) == 3
+    assert bench.linear_launches(8192, 5120, True) == 2
+    assert bench.linear_launches(8192, 5120, False) == 3
