@@ -117,6 +117,48 @@ def test_linear_short_k(nv, orc, m, k):
     assert nv.read_fault() == 0
 
 
+@pytest.mark.parametrize("case", ["zeros", "one_outlier", "tiny_and_huge", "zero_rows"])
+def test_linear_in_kernel_special_values(nv, orc, case):
+    """The in-kernel token quantization on X the quantizer's edge cases are
+    made of: all zeros (amax 0, g = 1), one huge outlier among N(0,1) values,
+    subnormal-range next to large magnitudes, and all-zero rows among
+    ordinary ones. The tokens' quantization equals nvfp4_quantize's bit for
+    bit (the same GEMM follows), and the oracle agrees within the tolerance
+    wherever the reference output is non-zero."""
+    m, k, n = 5, 1024, 256
+    x = gaussian(m, k, 77)
+    if case == "zeros":
+        x = torch.zeros((m, k), dtype=torch.bfloat16)
+    elif case == "one_outlier":
+        x[2, 517] = 3.0e4
+    elif case == "tiny_and_huge":
+        x[:, ::2] = x[:, ::2] * 1e-30
+        x[:, 1::64] = 6.0e4
+    else:
+        x[1] = 0.0
+        x[3] = 0.0
+    x = x.to(torch.bfloat16)
+    qw = orc.quantize(bits(gaussian(n, k, 78, 0.02)))
+    W = upload(qw)
+    xd = x.cuda()
+    for g in (None, torch.tensor([float(orc.global_from_amax(max(orc.tensor_amax(bits(x)), 1.0)))],
+                                 dtype=torch.float32, device="cuda")):
+        y = nv.linear(xd, W, out_dtype=torch.float32, global_scale=g,
+                      workspace=nv.linear_workspace(m, n, k))
+        gws = torch.empty(max(16, nv.gemm_workspace_bytes(m, n, k)), dtype=torch.uint8,
+                          device="cuda")
+        y2 = nv.gemm(nv.quantize(xd, global_scale=g), W, out_dtype=torch.float32, workspace=gws)
+        torch.cuda.synchronize()
+        assert torch.equal(y, y2), (case, g is None)
+        qx = orc.quantize(bits(x), None if g is None else np.float32(g.item()))
+        ref = orc.gemm(qx, qw)
+        if np.linalg.norm(ref) > 0:
+            gemm_check(y, ref, norms(orc, qx), norms(orc, qw), f"special {case}")
+        else:
+            assert float(y.abs().max()) == 0.0
+    assert nv.read_fault() == 0
+
+
 def test_linear_strided_and_ragged_x(nv, orc):
     """x with a row pitch larger than k, and k not a multiple of 256 (the last
     k-tile of every slice is partial): linear equals the chain."""
